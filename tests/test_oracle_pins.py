@@ -1,0 +1,464 @@
+"""Pins of the CPU oracle to facts fixed outside it (no GPU).
+
+Each test checks the oracle against something it does not share code with: numbers the
+pages state (tests/golden/pages_facts.json), library routines (scipy / statistics normal
+quantiles, numpy and torch 16-bit rounding), closed forms, invariants (monotonicity,
+power-of-two scale invariance, exact round trip), and brute force on small inputs
+(nearest level by exhaustive search, selection over all subsets).  The last tests plant
+mistakes in the oracle's inputs and check that the pins catch them.
+"""
+import itertools
+import json
+import math
+import os
+from statistics import NormalDist
+
+import numpy as np
+import pytest
+import torch
+from scipy.special import ndtri
+from scipy.stats import norm
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "pages_facts.json")
+FACTS = json.load(open(GOLDEN))
+
+
+def bits_of(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16).reshape(-1)
+
+
+def codes_of(packed: np.ndarray, n: int) -> np.ndarray:
+    c = np.stack([packed >> 4, packed & 15], axis=1).reshape(-1)
+    return c[:n].astype(np.int64)
+
+
+# ------------------------------------------------------------------ codebook
+
+
+def test_codebook_shape_and_anchors(book):
+    levels, mids = book
+    assert levels.size == FACTS["nf4_values"]["value"] == 16
+    assert levels[0] == -1.0 and levels[15] == 1.0
+    assert levels[7] == 0.0 and not np.signbit(levels[7])
+    assert np.all(np.diff(levels.astype(np.float64)) > 0)
+    # 7 negative levels, exact zero, 8 positive (asymmetric so that 0 and both ends exist)
+    assert (levels < 0).sum() == 7 and (levels > 0).sum() == 8
+    assert np.all((mids > levels[:-1]) & (mids < levels[1:]))
+
+
+def test_codebook_against_library_quantiles(book):
+    """Normal quantiles recomputed with scipy's ndtri and with statistics.NormalDist."""
+    levels, mids = book
+    pm = oracle.default_pmax()
+    assert pm == pytest.approx(1 - 0.5 * (1 / 32 + 1 / 30), abs=0)
+    pos = [ndtri(pm - k * (pm - 0.5) / 8) for k in range(8)]
+    neg = [-ndtri(pm - k * (pm - 0.5) / 7) for k in range(7)]
+    ref = np.array(sorted(pos + neg + [0.0])) / ndtri(pm)
+    assert np.array_equal(levels, ref.astype(np.float32))
+    nd = NormalDist()
+    ref2 = np.array(sorted([nd.inv_cdf(pm - k * (pm - 0.5) / 8) for k in range(8)]
+                           + [-nd.inv_cdf(pm - k * (pm - 0.5) / 7) for k in range(7)] + [0.0]))
+    ref2 /= nd.inv_cdf(pm)
+    assert np.max(np.abs(levels.astype(np.float64) - ref2)) < 2 ** -24
+    mref = ((levels[:-1].astype(np.float64) + levels[1:].astype(np.float64)) / 2).astype(np.float32)
+    assert np.array_equal(mids, mref)
+
+
+def test_codebook_equal_probability_spacing(book):
+    """Each half's levels sit at evenly spaced normal probabilities ("equal share")."""
+    levels, _ = book
+    z = ndtri(oracle.default_pmax())
+    p = norm.cdf(levels.astype(np.float64) * z)
+    assert np.allclose(np.diff(p[:8]), np.diff(p[:8]).mean(), rtol=0, atol=1e-7)
+    assert np.allclose(np.diff(p[7:]), np.diff(p[7:]).mean(), rtol=0, atol=1e-7)
+    assert p[0] == pytest.approx(1 - oracle.default_pmax(), abs=1e-7)
+    assert p[15] == pytest.approx(oracle.default_pmax(), abs=1e-7)
+
+
+def test_codebook_histogram_roughly_flat(book):
+    """Normal samples at the codebook's own scale land nearly evenly on the 16 values."""
+    _, mids = book
+    z = ndtri(oracle.default_pmax())
+    x = np.random.default_rng(0).standard_normal(400_000) / z
+    h = np.bincount(np.searchsorted(mids.astype(np.float64), x, side="left"), minlength=16)
+    r = h / h.mean()
+    assert r.min() > 0.8 and r.max() < 1.2, r
+
+
+def test_codebook_rejects_bad_pmax():
+    for bad in (0.5, 1.0, 0.2, 1.5):
+        with pytest.raises(ValueError):
+            oracle.codebook(bad)
+
+
+# ---------------------------------------------------------------- conversions
+
+
+def test_dtype_decode_all_bit_patterns():
+    allbits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    f16 = oracle.dtype_bits_to_f32(allbits, oracle.F16)
+    ref16 = allbits.view(np.float16).astype(np.float32)
+    same = (f16.view(np.uint32) == ref16.view(np.uint32)) | (np.isnan(f16) & np.isnan(ref16))
+    assert same.all()
+    bf = oracle.dtype_bits_to_f32(allbits, oracle.BF16)
+    refb = torch.from_numpy(allbits.view(np.int16)).view(torch.bfloat16).float().numpy()
+    same = (bf.view(np.uint32) == refb.view(np.uint32)) | (np.isnan(bf) & np.isnan(refb))
+    assert same.all()
+
+
+@pytest.mark.parametrize("dtype", [oracle.F16, oracle.BF16])
+def test_dtype_rounding_matches_libraries(dtype):
+    rng = np.random.default_rng(1)
+    parts = [rng.standard_normal(20000).astype(np.float32) * s for s in (1e-8, 1e-5, 0.02, 3, 7e4)]
+    # ties and their neighbours: halfway points between adjacent 16-bit values
+    base = rng.standard_normal(4000).astype(np.float32)
+    if dtype == oracle.F16:
+        lo = base.astype(np.float16).astype(np.float32)
+    else:
+        lo = torch.from_numpy(base).to(torch.bfloat16).float().numpy()
+    hi = np.nextafter(lo, np.float32(np.inf) * np.sign(lo + 1e-30))
+    parts += [lo, (lo.astype(np.float64) + 2.0 ** -30).astype(np.float32), hi]
+    if dtype == oracle.BF16:
+        parts.append(np.array([3.3e38, -3.39e38, 1e-39, -2e-40, 0.0, -0.0], np.float32))
+    else:
+        parts.append(np.array([65519.0, 65520.0, -70000.0, 6e-8, 3e-8, 2.9e-8, -0.0], np.float32))
+    x = np.concatenate(parts)
+    got = oracle.f32_to_dtype_bits(x, dtype)
+    if dtype == oracle.F16:
+        with np.errstate(over="ignore"):
+            ref = x.astype(np.float16).view(np.uint16)
+    else:
+        ref = bits_of(torch.from_numpy(x).to(torch.bfloat16))
+    assert np.array_equal(got, ref)
+
+
+# ---------------------------------------------------------------- quantize
+
+
+def _nearest_level_bruteforce(v64: np.ndarray, levels: np.ndarray) -> np.ndarray:
+    d = np.abs(v64[:, None] - levels.astype(np.float64)[None, :])
+    return np.argmin(d, axis=1)  # argmin takes the first (lower) index on ties
+
+
+def _normalized(x32: np.ndarray, a: float) -> np.ndarray:
+    r = np.float32(1.0) / np.float32(a)
+    return (x32 * r).astype(np.float32)
+
+
+@pytest.mark.parametrize("dtype", [oracle.F16, oracle.BF16])
+def test_codes_equal_nearest_level_bruteforce(book, dtype):
+    levels, mids = book
+    rng = np.random.default_rng(7)
+    tdt = torch.float16 if dtype == oracle.F16 else torch.bfloat16
+    w = torch.from_numpy(
+        np.concatenate([rng.standard_normal(64 * 300), rng.standard_t(3, 64 * 200),
+                        rng.uniform(-1, 1, 64 * 100)]).astype(np.float32) * 0.02).to(tdt)
+    bits = bits_of(w)
+    packed, absmax, nonfinite = oracle.quantize(bits, dtype)
+    assert not nonfinite
+    codes = codes_of(packed, bits.size)
+    x = w.float().numpy()
+    # the oracle's absmax is the plain max |x| per block
+    assert np.array_equal(absmax, np.abs(x).reshape(-1, 64).max(axis=1))
+    v = np.concatenate([_normalized(xb, a) for xb, a in zip(x.reshape(-1, 64), absmax)])
+    brute = _nearest_level_bruteforce(v.astype(np.float64), levels)
+    diff = codes != brute
+    # the midpoint rule and exhaustive search may only differ within 1 ulp of a midpoint
+    if diff.any():
+        vv = v[diff]
+        gap = np.min(np.abs(vv[:, None].astype(np.float64) - mids.astype(np.float64)[None, :]), axis=1)
+        assert np.all(gap <= np.spacing(np.abs(vv)) * 1.0), (vv, gap)
+    assert diff.sum() <= 2
+
+
+@pytest.mark.parametrize("dtype", [oracle.F16, oracle.BF16])
+def test_round_trip_on_scaled_levels(book, dtype):
+    """Weights equal to dtype(level * a), with a present, come back exactly: error 0."""
+    levels, _ = book
+    rng = np.random.default_rng(3)
+    tdt = torch.float16 if dtype == oracle.F16 else torch.bfloat16
+    nblk = 64
+    codes = rng.integers(0, 16, size=(nblk, 64))
+    codes[:, 5] = rng.choice([0, 15], size=nblk)  # absmax element (|level| = 1)
+    a = torch.from_numpy(rng.uniform(0.001, 0.5, nblk).astype(np.float32)).to(tdt).float().numpy()
+    prod = (levels[codes] * a[:, None]).astype(np.float32)
+    w = torch.from_numpy(prod.reshape(-1)).to(tdt)
+    bits = bits_of(w)
+    packed, absmax, _ = oracle.quantize(bits, dtype)
+    assert np.array_equal(absmax, a)
+    assert np.array_equal(codes_of(packed, bits.size), codes.reshape(-1))
+    # the packed layout: even element in the high nibble
+    c = codes.reshape(-1)
+    assert np.array_equal(packed, ((c[0::2] << 4) | c[1::2]).astype(np.uint8))
+    se, sw, rel = oracle.layer_error(bits, dtype)
+    assert se == 0.0 and rel == 0.0 and sw > 0
+    back = oracle.dequantize(packed, bits.size, dtype, absmax=absmax)
+    assert np.array_equal(back, bits)
+
+
+def test_zero_block_and_ragged_tail(book):
+    w = np.zeros(65, np.float16)
+    w[64] = 0.5
+    packed, absmax, _ = oracle.quantize(w, oracle.F16)
+    assert packed.size == 33 and absmax.size == 2
+    assert np.all(packed[:32] == 0x77)
+    assert absmax[0] == 0.0 and absmax[1] == 0.5
+    assert packed[32] == 0xF0  # code 15 in the high nibble, low nibble left 0
+    se, sw, rel = oracle.layer_error(np.zeros(100, np.float16), oracle.F16)
+    assert (se, sw, rel) == (0.0, 0.0, 0.0)
+
+
+def test_codes_monotone_in_x(book):
+    rng = np.random.default_rng(11)
+    x = np.sort(rng.standard_normal((50, 64)).astype(np.float16), axis=1)
+    packed, _, _ = oracle.quantize(x.reshape(-1), oracle.F16)
+    c = codes_of(packed, x.size).reshape(50, 64)
+    assert np.all(np.diff(c, axis=1) >= 0)
+
+
+@pytest.mark.parametrize("k", [-9, -1, 3, 20])
+def test_power_of_two_scale_invariance(k):
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal(64 * 40) * 0.02).astype(np.float32)
+    w = torch.from_numpy(x).to(torch.bfloat16)
+    ws = (w.float() * 2.0 ** k).to(torch.bfloat16)  # exact: power of two, no range issue
+    assert torch.equal(ws.float() / 2.0 ** k, w.float())
+    p1, a1, _ = oracle.quantize(bits_of(w), oracle.BF16)
+    p2, a2, _ = oracle.quantize(bits_of(ws), oracle.BF16)
+    assert np.array_equal(p1, p2)
+    assert np.array_equal(a2, (a1 * 2.0 ** k).astype(np.float32))
+    r1 = oracle.layer_error(bits_of(w), oracle.BF16)[2]
+    r2 = oracle.layer_error(bits_of(ws), oracle.BF16)[2]
+    assert r1 == r2
+
+
+def test_subnormal_absmax_block_is_scale_invariant():
+    """A bf16 block below the fp32 normal range codes like the same block scaled by 2^100."""
+    rng = np.random.default_rng(9)
+    x = (rng.standard_normal(64 * 8) * 1e-39).astype(np.float32)
+    w = torch.from_numpy(x).to(torch.bfloat16)
+    big = (w.double() * 2.0 ** 100).to(torch.bfloat16)
+    assert torch.equal((big.double() / 2.0 ** 100).to(torch.bfloat16), w)
+    p1, a1, _ = oracle.quantize(bits_of(w), oracle.BF16)
+    p2, _, _ = oracle.quantize(bits_of(big), oracle.BF16)
+    assert np.all(a1 < 2.0 ** -126)
+    assert np.array_equal(p1, p2)
+
+
+def test_nonfinite_inputs_flagged():
+    w = np.zeros(200, np.float16)
+    w[3] = np.nan
+    w[100] = np.inf
+    packed, absmax, nonfinite = oracle.quantize(w, oracle.F16)
+    assert nonfinite and np.isnan(absmax[0]) and np.isinf(absmax[1])
+    assert math.isnan(oracle.layer_error(w, oracle.F16)[2])
+
+
+# ---------------------------------------------------------------- score
+
+
+@pytest.mark.parametrize("dtype", [oracle.F16, oracle.BF16])
+def test_layer_error_matches_bruteforce_reconstruction(book, dtype):
+    levels, _ = book
+    rng = np.random.default_rng(21)
+    tdt = torch.float16 if dtype == oracle.F16 else torch.bfloat16
+    n = 64 * 97 + 13
+    w = torch.from_numpy((rng.standard_t(4, n) * 0.01).astype(np.float32)).to(tdt)
+    bits = bits_of(w)
+    x = w.double().numpy()
+    nb = (n + 63) // 64
+    se = 0.0
+    for b in range(nb):
+        xb = w.float().numpy()[64 * b: 64 * b + 64]
+        a = np.float32(np.abs(xb).max())
+        v = _normalized(xb, a)
+        c = _nearest_level_bruteforce(v.astype(np.float64), levels)
+        what = torch.from_numpy((levels[c] * a).astype(np.float32)).to(tdt).double().numpy()
+        se += float(np.sum((x[64 * b: 64 * b + 64] - what) ** 2))
+    o_se, o_sw, o_rel = oracle.layer_error(bits, dtype)
+    assert o_sw == pytest.approx(float(np.sum(x * x)), rel=1e-13)
+    assert o_se == pytest.approx(se, rel=1e-12)
+    assert o_rel == pytest.approx(math.sqrt(se / float(np.sum(x * x))), rel=1e-6)
+
+
+def test_heavy_tailed_layers_rank_first_on_tiny():
+    from quantized_lora_setup_b200 import synth
+    wl = synth.tiny(0)
+    rel, cost = [], []
+    for i, spec in enumerate(wl.layers):
+        w = synth.layer_host(spec, wl.seed, i)
+        rel.append(oracle.layer_error(bits_of(w), oracle.F16)[2])
+        cost.append(oracle.cost_bytes(spec.numel))
+    heavy = sorted(i for i, s in enumerate(wl.layers) if s.dist == "t")
+    sel = oracle.select_topk(rel, cost, wl.budgets[0], wl.k_cap)
+    assert sorted(sel) == heavy
+    normal = [r for i, r in enumerate(rel) if i not in heavy]
+    assert min(rel[i] for i in heavy) > 1.05 * max(normal)
+
+
+# ---------------------------------------------------------------- double quantization
+
+
+def test_dq_saving_matches_page_figure():
+    n = 64 * 256 * 10
+    absmax = np.random.default_rng(0).uniform(0, 1, n // 64).astype(np.float32)
+    codes8, scales, _ = oracle.double_quant(absmax)
+    bits_dq = (codes8.nbytes + scales.nbytes) * 8 / n
+    bits_plain = absmax.nbytes * 8 / n
+    saving = bits_plain - bits_dq
+    assert saving == 0.5 - (8 / 64 + 32 / (64 * 256)) == 0.373046875
+    fact = FACTS["dq_saving_bits_per_param"]
+    assert round(saving, fact["decimals"]) == fact["value"]
+
+
+def test_dq_special_cases():
+    s = np.float32(0.37)
+    a = np.array([s] * 256 + [0.0, s / 2, s] + [0.0] * 253 + [0.0] * 10, np.float32)
+    codes8, scales, nf = oracle.double_quant(a)
+    assert not nf
+    assert np.all(codes8[:256] == 255) and scales[0] == s
+    assert list(codes8[256:259]) == [0, 128, 255]  # 127.5 rounds to the even 128
+    assert scales[2] == 0.0 and np.all(codes8[512:] == 0)
+    back = oracle.dequantize(np.zeros(128, np.uint8), 256, oracle.F16, codes8=codes8[:4],
+                             scales=scales[:1])
+    assert back.size == 256
+    a2 = np.array([1.0, np.nan], np.float32)
+    _, sc2, nf2 = oracle.double_quant(a2)
+    assert nf2 and np.isnan(sc2[0])
+
+
+def test_dq_codes_equal_bruteforce_nearest():
+    rng = np.random.default_rng(4)
+    a = np.abs(rng.standard_normal(256 * 37 + 5)).astype(np.float32) * 0.05
+    codes8, scales, _ = oracle.double_quant(a)
+    for d in range(scales.size):
+        blk = a[256 * d: 256 * d + 256].astype(np.float64)
+        s = float(scales[d])
+        assert s == blk.max()
+        grid = np.arange(256) / 255.0 * s
+        brute = np.argmin(np.abs(blk[:, None] - grid[None, :]), axis=1)
+        got = codes8[256 * d: 256 * d + blk.size]
+        diff = got != brute
+        assert diff.sum() <= 1  # only within one rounding of a half-way point
+        if diff.any():
+            frac = blk[diff] / s * 255
+            assert np.all(np.abs(frac - np.floor(frac) - 0.5) < 1e-5)
+
+
+def test_dequant_with_exact_dq_equals_plain_absmax(book):
+    """Constants that double-quantize exactly (code 255) dequantize like the raw absmax."""
+    rng = np.random.default_rng(8)
+    w = torch.from_numpy((rng.standard_normal(256 * 64) * 0.02).astype(np.float32)).to(torch.bfloat16)
+    bits = bits_of(w)
+    packed, absmax, _ = oracle.quantize(bits, oracle.BF16)
+    flat = np.full_like(absmax, absmax.max())
+    codes8, scales, _ = oracle.double_quant(flat)
+    assert np.all(codes8 == 255)
+    d1 = oracle.dequantize(packed, bits.size, oracle.BF16, codes8=codes8, scales=scales)
+    d2 = oracle.dequantize(packed, bits.size, oracle.BF16, absmax=flat)
+    assert np.array_equal(d1, d2)
+
+
+def test_dequant_reconstructs_layer_error(book):
+    """The error the score reports is the error of the dequantized weights."""
+    rng = np.random.default_rng(12)
+    n = 64 * 33 + 7
+    w = torch.from_numpy((rng.standard_normal(n) * 0.03).astype(np.float32)).to(torch.float16)
+    bits = bits_of(w)
+    packed, absmax, _ = oracle.quantize(bits, oracle.F16)
+    deq = oracle.dequantize(packed, n, oracle.F16, absmax=absmax).view(np.float16).astype(np.float64)
+    x = w.double().numpy()
+    se, sw, _ = oracle.layer_error(bits, oracle.F16)
+    assert se == pytest.approx(float(np.sum((x - deq) ** 2)), rel=1e-12)
+
+
+# ---------------------------------------------------------------- selection
+
+
+def _bruteforce_select(e, cost, budget, k_cap):
+    L = len(e)
+
+    def before(j, i):
+        if math.isnan(e[j]) != math.isnan(e[i]):
+            return math.isnan(e[i])
+        if not math.isnan(e[j]) and e[j] != e[i]:
+            return e[j] > e[i]
+        return j < i
+
+    best = ()
+    for r in range(L + 1):
+        for S in itertools.combinations(range(L), r):
+            s = set(S)
+            if k_cap >= 0 and len(s) > k_cap:
+                continue
+            if sum(cost[i] for i in s) > budget:
+                continue
+            closed = all(not before(j, i) for i in s for j in range(L) if j not in s)
+            if closed and len(s) > len(best):
+                best = S
+    return sorted(best)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_select_equals_bruteforce_over_subsets(seed):
+    rng = np.random.default_rng(seed)
+    L = int(rng.integers(1, 11))
+    e = rng.choice([0.05, 0.1, 0.1, 0.2, 0.3, float("nan")], size=L).astype(np.float32)
+    e = np.where(rng.uniform(size=L) < 0.5, rng.uniform(0, 1, L).astype(np.float32), e)
+    cost = rng.integers(1, 100, L)
+    budget = int(rng.integers(0, 300))
+    k_cap = int(rng.choice([-1, 0, 1, 2, 5]))
+    got = oracle.select_topk(e, cost, budget, k_cap)
+    assert sorted(got) == _bruteforce_select(list(map(float, e)), list(cost), budget, k_cap)
+
+
+def test_select_rules():
+    e = [0.3, 0.5, 0.5, float("nan"), 0.1]
+    assert oracle.select_topk(e, [1] * 5, 100) == [1, 2, 0, 4, 3]  # ties by index, NaN last
+    assert oracle.select_topk(e, [1] * 5, 100, k_cap=2) == [1, 2]
+    assert oracle.select_topk(e, [1] * 5, 0) == []
+    # walking the ranking stops at the first layer that does not fit
+    assert oracle.select_topk([0.9, 0.8, 0.7], [5, 10, -8], 8) == [0]
+    with pytest.raises(ValueError):
+        oracle.select_topk(e, [1] * 5, -1)
+
+
+def test_cost_bytes_closed_form():
+    for n in (1, 7, 64, 65, 4096 * 4096, 11008 * 4096, 16385):
+        nb = -(-n // 64)
+        assert oracle.cost_bytes(n) == 2 * n - (-(-n // 2) + nb + 4 * -(-nb // 256))
+    # the 0.2 GiB quality-setting budget keeps a few 4096x4096 layers
+    per = oracle.cost_bytes(4096 * 4096)
+    assert int(FACTS["quality_setting_extra_memory_gib"]["value"] * 2 ** 30) // per == 8
+
+
+# ---------------------------------------------------------------- planted mistakes
+
+
+def test_pins_catch_a_reversed_codebook(book):
+    levels, mids = book
+    wrong = (-levels[::-1].copy(), -mids[::-1].copy())  # a plausible sign slip
+    rng = np.random.default_rng(3)
+    codes = rng.integers(0, 16, size=(8, 64))
+    codes[:, 0] = 15
+    a = np.float32(0.25)
+    w = torch.from_numpy((levels[codes] * a).astype(np.float32).reshape(-1)).to(torch.float16)
+    se, _, _ = oracle.layer_error(bits_of(w), oracle.F16, book=wrong)
+    assert se > 0  # the round-trip pin would fail
+
+
+def test_pins_catch_thresholds_off_by_one_index(book):
+    levels, mids = book
+    wrong = (levels, levels[1:].copy())  # thresholds at q[j+1] instead of the midpoints
+    rng = np.random.default_rng(7)
+    w = torch.from_numpy((rng.standard_normal(64 * 50) * 0.02).astype(np.float32)).to(torch.float16)
+    bits = bits_of(w)
+    p_ok, a_ok, _ = oracle.quantize(bits, oracle.F16)
+    p_bad, _, _ = oracle.quantize(bits, oracle.F16, book=wrong)
+    x = w.float().numpy()
+    v = np.concatenate([_normalized(xb, a) for xb, a in zip(x.reshape(-1, 64), a_ok)])
+    brute = _nearest_level_bruteforce(v.astype(np.float64), levels)
+    assert np.array_equal(codes_of(p_ok, bits.size), brute)
+    assert not np.array_equal(codes_of(p_bad, bits.size), brute)
