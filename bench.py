@@ -1,0 +1,458 @@
+#!/usr/bin/env python
+"""Benchmark of the NF4 scoring pass (the AQLoRA setup pass) on B200.
+
+One step = one pass of the whole path over a model's weights, resident in HBM:
+fused NF4 quantize + nibble pack + double quantization + per-layer reconstruction error
+for every layer (aqnf4_layer_error), then the top-K selection under the byte budget
+(aqnf4_select_topk).  With N ranks the layers are split by LPT and the scores are
+all-gathered before the selection.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle instead, on a
+bounded sample of the same workload, on this machine's host cores.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+from concurrent.futures import ThreadPoolExecutor
+from datetime import timedelta
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "NF4 quantize+score GB/s (fp16 weights read) and % of HBM roofline; dequant GB/s"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SRC = os.path.join(ROOT, "quantized_lora_setup_b200", "csrc", "quant_score.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "k_quant_score_7b.md")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default="7b", choices=["tiny", "1.4b", "7b", "14b"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dequant", action="store_true")
+    return ap.parse_args()
+
+
+def host_threads() -> int:
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    return max(1, min(n, 64))
+
+
+def workload_desc(wl) -> str:
+    shapes = sorted({(s.rows, s.cols) for s in wl.layers})
+    sh = ", ".join(f"{r}x{c}" for r, c in shapes)
+    dts = sorted({str(s.dtype).replace("torch.", "") for s in wl.layers})
+    return (f"{wl.name}-shaped: {len(wl.layers)} linear layers ({sh}), {'/'.join(dts)}, "
+            f"{wl.numel / 1e9:.3f}e9 weights, synthetic seeded")
+
+
+def algorithmic_bytes(n: int) -> int:
+    """Bytes the fused pass must move for an n-element layer: read the 16-bit weights,
+    write packed nibbles, 8-bit DQ codes and fp32 DQ scales."""
+    nb = (n + 63) // 64
+    return 2 * n + (n + 1) // 2 + nb + 4 * ((nb + 255) // 256)
+
+
+# ------------------------------------------------------------------ CPU oracle leg
+
+
+def oracle_pass(sample):
+    """The oracle's version of one step on a list of (bits, dtype) layer samples."""
+    import oracle
+
+    def one(item):
+        b, dt = item
+        _, absmax, _ = oracle.quantize(b, dt)
+        oracle.double_quant(absmax)
+        oracle.layer_error(b, dt)
+        return b.size
+
+    with ThreadPoolExecutor(max_workers=len(sample)) as ex:
+        return sum(ex.map(one, sample))
+
+
+def build_oracle_sample(wl, threads, per_thread_elems, layer_tensors=None):
+    """One slice per thread: the first elements of the workload's first `threads` layers."""
+    from quantized_lora_setup_b200 import synth
+    import oracle
+    sample = []
+    for i in range(min(threads, len(wl.layers))):
+        spec = wl.layers[i]
+        if layer_tensors is not None:
+            w = layer_tensors[i].reshape(-1)[: min(spec.numel, per_thread_elems)].cpu()
+        else:
+            w = synth.layer_host(spec, wl.seed, i).reshape(-1)[: min(spec.numel, per_thread_elems)]
+        dt = oracle.BF16 if str(w.dtype) == "torch.bfloat16" else oracle.F16
+        n = (w.numel() // 16384) * 16384 or w.numel()
+        sample.append((synth.bits_u16(w[:n]), dt))
+    return sample
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from quantized_lora_setup_b200 import synth
+    wl = synth.workload(args.workload)
+    threads = host_threads()
+    # ~75 ns per element per thread for quantize + DQ + error in the oracle: size each step so
+    # the whole run (warm-up + steps) stays near two minutes.
+    per_step_s = max(0.2, 120.0 / max(1, args.steps + args.warmup))
+    per_thread = max(16384, int(per_step_s / 75e-9) // 16384 * 16384)
+    sample = build_oracle_sample(wl, threads, per_thread)
+    elems = sum(b.size for b, _ in sample)
+    for _ in range(args.warmup):
+        oracle_pass(sample)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_pass(sample)
+    dt = time.perf_counter() - t0
+    value = 2 * elems * args.steps / dt / 1e9
+    desc = (f"{len(sample)} slices of up to {per_thread} elements (the first elements of the "
+            f"first {len(sample)} layers), {elems} weights per step, one thread per slice")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": workload_desc(wl), "sample": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": len(sample), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ clocks
+
+
+class ClockSampler:
+    """Polls NVML every 10 ms (SM clock, max SM clock, clock-event reasons) in a thread."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int):
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            try:  # CUDA and NVML may number the GPUs differently: match by UUID
+                uuid = str(torch.cuda.get_device_properties(index).uuid)
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(
+                    uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: report no clocks rather than fail the bench
+            self.nv, self.err = None, str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            self._stop.wait(0.01)
+
+    def start(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+
+    def summary(self):
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": self.err}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ native arm
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic():
+    """Per-launch DRAM bytes of k_quant_score from the committed ncu summary, if it was
+    taken on the current kernel source (its sha256 is recorded beside the number)."""
+    try:
+        text = open(TRAFFIC_FILE).read()
+        src = hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith(("traffic_bytes_per_launch", "source_sha256")):
+            k, v = line.split(":", 1)
+            vals[k.strip().strip("`- ")] = v.strip().strip("` ")
+    if vals.get("source_sha256") != src:
+        return None
+    try:
+        return float(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def run_native(args):
+    import torch
+    import torch.distributed as dist
+
+    from quantized_lora_setup_b200 import aqnf4, synth
+    from quantized_lora_setup_b200.shard import ScoreGather, lpt_partition
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    aqnf4.library()
+
+    wl = synth.workload(args.workload)
+    L = len(wl.layers)
+    parts = lpt_partition([s.numel for s in wl.layers], world)
+    mine = parts[rank]
+    weights = [synth.layer_device(wl.layers[i], wl.seed, i, dev) for i in mine]
+    stor = [aqnf4.NF4Storage(w.numel(), dev) for w in weights]
+    descs = aqnf4.make_layers([{"w": w, "packed": s.packed, "codes8": s.codes8,
+                                "scales": s.scales} for w, s in zip(weights, stor)])
+    ws = torch.empty(max(256, aqnf4.aqnf4_workspace_size(descs)), dtype=torch.uint8, device=dev)
+    se = torch.empty(max(1, len(mine)), dtype=torch.float64, device=dev)
+    sw = torch.empty_like(se)
+    rel = torch.empty(max(1, len(mine)), dtype=torch.float32, device=dev)
+    cost = torch.tensor([aqnf4.aqnf4_cost_bytes(s.numel) for s in wl.layers], dtype=torch.int64,
+                        device=dev)
+    sel = torch.empty(L, dtype=torch.int32, device=dev)
+    kout = torch.empty(1, dtype=torch.int32, device=dev)
+    budget = wl.budgets[0]
+    gather = ScoreGather(parts, rank, L, dev) if world > 1 else None
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev_a=None, ev_b=None):
+        if ev_a is not None:
+            ev_a.record(stream)
+        if mine:
+            aqnf4.aqnf4_layer_error(descs, ws, se, sw, rel, None, stream)
+        if ev_b is not None:
+            ev_b.record(stream)
+        scores = gather(rel) if gather is not None else rel
+        aqnf4.aqnf4_select_topk(scores, cost, budget, wl.k_cap, sel, kout, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = aqnf4.aqnf4_launch_count()
+    clocks.start()
+    t_start.record(stream)
+    for i in range(K):
+        step(*ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.stop()
+    launches = aqnf4.aqnf4_launch_count() - launches0
+    barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    kern_ms = [a.elapsed_time(b) for a, b in ev]
+    agg = torch.tensor([elapsed_ms, float(launches)], dtype=torch.float64, device=dev)
+    if world > 1:
+        mx = agg[:1].clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        tot = agg[1:].clone()
+        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
+        elapsed_ms, launches = float(mx.item()), int(tot.item())
+    total_weight_bytes = wl.weight_bytes
+    value = total_weight_bytes * K / (elapsed_ms / 1e3) / 1e9
+
+    # roofline of the dominant kernel (this rank's fused pass; the small finalize kernel
+    # that follows it is inside the same event pair, so this slightly understates it)
+    my_alg = sum(algorithmic_bytes(w.numel()) for w in weights)
+    kern_avg_ms = statistics.mean(kern_ms)
+    achieved = my_alg / (kern_avg_ms / 1e3) / 1e9
+    peak, peak_src = measured_hbm_peak()
+    traffic = recorded_traffic()
+
+    k_sel = int(kout.item())
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": max(3, args.warmup), "ms_per_step": elapsed_ms / K, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {
+            "workload": workload_desc(wl), "layers": L, "weight_bytes": total_weight_bytes,
+            "budget_bytes": budget, "k_cap": wl.k_cap,
+            "l2": "inputs larger than L2 (weights read once per step, no flush needed)",
+            "parallelism": f"layers split over {world} rank(s) by LPT; scores all-gathered"
+            if world > 1 else "single GPU",
+            "outputs": "packed NF4 + 8-bit DQ codes + fp32 DQ scales + per-layer scores",
+        },
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic, "kernel": "k_quant_score",
+                     "peak_source": f"{peak_src} hbm_gbs", "alg_bytes_per_launch": my_alg,
+                     "launch_ms": kern_avg_ms},
+        "clocks": clocks.summary(),
+        "gpu_launches": launches,
+        "selected": {"k": k_sel, "of": L},
+    }
+
+    if not args.no_dequant:
+        result["dequant"] = bench_dequant(dev, stream, peak)
+
+    if not args.no_e2e:
+        result["e2e"] = bench_e2e(args, weights, step, sel, kout, dev, stream, world,
+                                  total_weight_bytes, L)
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = host_threads()
+        per_thread = max(16384, int(20.0 / threads / 75e-9) // 16384 * 16384)
+        sample = build_oracle_sample(wl, threads, per_thread, layer_tensors=weights)
+        t0 = time.perf_counter()
+        elems = oracle_pass(sample)
+        dt = time.perf_counter() - t0
+        result["cpu_baseline"] = {
+            "value": 2 * elems / dt / 1e9, "unit": UNIT, "cores": len(sample), "kind": "oracle",
+            "sample": f"{len(sample)} slices of up to {per_thread} elements from the first "
+                      f"{len(sample)} layers ({elems} weights), quantize + DQ + error, one "
+                      f"thread per slice"}
+
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+def bench_dequant(dev, stream, peak):
+    """Standalone NF4+DQ -> bf16 dequantization of a 28672x8192 matrix; four distinct
+    inputs rotate so the 117 MB packed input cannot stay in the 126 MB L2."""
+    import torch
+
+    from quantized_lora_setup_b200 import aqnf4, synth
+    rows, cols = synth.DEQUANT_SHAPES[-1]
+    n = rows * cols
+    inputs = []
+    for s in range(4):
+        w = synth.normal_matrix_device(rows, cols, seed=1000 + s, device=dev)
+        st = aqnf4.NF4Storage(n, dev)
+        aqnf4.score_layers([w], [st])
+        del w
+        inputs.append(st)
+    out = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    for st in inputs:
+        aqnf4.aqnf4_dequantize(st.packed, st.codes8, st.scales, None, n, out, stream)
+    reps = 40
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    a.record(stream)
+    for i in range(reps):
+        st = inputs[i % 4]
+        aqnf4.aqnf4_dequantize(st.packed, st.codes8, st.scales, None, n, out, stream)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b) / reps
+    nb = (n + 63) // 64
+    alg = n // 2 + nb + 4 * ((nb + 255) // 256) + 2 * n
+    gbs = alg / (ms / 1e3) / 1e9
+    return {"shape": f"{rows}x{cols}", "ms_per_launch": ms, "value": gbs, "unit": "GB/s",
+            "out_gbs": 2 * n / (ms / 1e3) / 1e9,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                         "frac": gbs / peak, "traffic": None, "kernel": "k_dequant",
+                         "alg_bytes_per_launch": alg}}
+
+
+def bench_e2e(args, weights, step, sel, kout, dev, stream, world, total_weight_bytes, L):
+    """The same step through the public API with the weights starting in pinned host
+    memory: every step copies them in, runs the pass and reads the selection back."""
+    import torch
+    import torch.distributed as dist
+
+    host = [torch.empty(w.shape, dtype=w.dtype, pin_memory=True) for w in weights]
+    for h, w in zip(host, weights):
+        h.copy_(w)
+    steps = max(1, min(args.steps, 5))
+    res_k = torch.empty(1, dtype=torch.int32, pin_memory=True)
+    res_sel = torch.empty(L, dtype=torch.int32, pin_memory=True)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    a.record(stream)
+    for _ in range(steps):
+        for h, w in zip(host, weights):
+            w.copy_(h, non_blocking=True)
+        step()
+        res_k.copy_(kout, non_blocking=True)
+        res_sel.copy_(sel, non_blocking=True)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    h2d = sum(w.numel() * w.element_size() for w in weights)
+    return {"value": total_weight_bytes * steps / (ms / 1e3) / 1e9, "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4 + 4 * L, "steps": steps}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,181 @@
+/*
+ * aqnf4.h -- C ABI of libaqnf4: the per-layer NF4 pass on NVIDIA B200 (sm_100a).
+ *
+ * The pass quantizes each linear layer of a model to 4-bit NormalFloat (NF4) in blocks of
+ * 64 elements, double-quantizes the per-block absmax constants to 8 bits in blocks of 256,
+ * measures each layer's relative reconstruction error, and keeps the top-K layers in 16 bits
+ * under a byte budget.  A standalone NF4 -> 16-bit dequantization comes with it.
+ *
+ * Sources (page title, section):
+ *   "QLoRA" (ai360xpert.com), "How It Works": NF4 spreads the weights evenly over its 16
+ *       values; double quantization quantizes the quantization constants (about 0.37 bits
+ *       per parameter saved); weights are dequantized to 16 bits on the fly.
+ *   "QLoRA Explained" (devtoolshub.net), "NF4", "Double Quantization".
+ *   arxivdaily 2608.23816, "English abstract": one pass over the weights ranks layers by
+ *       NF4 reconstruction error and keeps the top-K in fp16 under a memory budget.
+ *   "AQLoRA: A Zero-Search Recipe for Fast Quantized LoRA Fine-Tuning", "Technical Details":
+ *       every layer is ranked; the memory budget is configurable.
+ *
+ * Conventions for every call:
+ *   - The caller owns every buffer.  The library allocates nothing and frees nothing.
+ *   - Pointers named "device" must be CUDA device (or managed) memory of the current device.
+ *   - Calls with a stream argument are asynchronous on that stream (0 = legacy default
+ *     stream).  The returned status covers the synchronous argument checks and the launch;
+ *     data-dependent conditions are reported through a device flag word (below).
+ *   - dev_flag (optional, device int32): when any input element is NaN or infinite the
+ *     kernels store AQNF4_ERR_NONFINITE there; nothing is stored otherwise, so the caller
+ *     zeroes it before the call and reads it after synchronizing.  The outputs of such a
+ *     block are still written (see aqnf4_quantize) but are not meaningful.
+ *   - 16-bit weights are either IEEE binary16 (AQNF4_F16) or bfloat16 (AQNF4_BF16).
+ *   - Layout of the NF4 data of an n-element tensor (flattened row-major):
+ *       packed  uint8[ceil(n/2)]   byte i = code[2i] << 4 | code[2i+1]; an odd n leaves the
+ *                                  low nibble of the last byte 0.
+ *       absmax  float[ceil(n/64)]  max |x| of each 64-element block (the last may be short).
+ *       codes8  uint8[ceil(n/64)]  double-quantized absmax, see aqnf4_double_quant.
+ *       scales  float[ceil(ceil(n/64)/256)]
+ *   - Codes index the ascending 16-level codebook returned by aqnf4_codebook; code 7 is the
+ *     exact zero.
+ */
+#ifndef AQNF4_H
+#define AQNF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* cudaStream_t;
+
+#if defined(__GNUC__)
+#define AQNF4_API __attribute__((visibility("default")))
+#else
+#define AQNF4_API
+#endif
+
+typedef enum {
+  AQNF4_OK = 0,
+  AQNF4_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, bad count or budget */
+  AQNF4_ERR_ALIGNMENT = 2,   /* a pointer lacks the alignment stated for it */
+  AQNF4_ERR_DTYPE = 3,       /* dtype is neither AQNF4_F16 nor AQNF4_BF16 */
+  AQNF4_ERR_NONFINITE = 4,   /* (device flag only) an input element is NaN or infinite */
+  AQNF4_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
+  AQNF4_ERR_TIMEOUT = 6,     /* (device flag only) a bounded wait inside a kernel ran out */
+  AQNF4_ERR_WORKSPACE = 7    /* workspace missing, misaligned or smaller than required */
+} aqnf4_status;
+
+typedef enum { AQNF4_F16 = 0, AQNF4_BF16 = 1 } aqnf4_dtype;
+
+/* One linear layer for aqnf4_layer_error.  All pointers are device pointers.
+   w      : numel 16-bit weights, 16-byte aligned (required).
+   packed : optional output, ceil(numel/2) bytes, 16-byte aligned.
+   absmax : optional output, ceil(numel/64) floats, 4-byte aligned.
+   codes8 : optional output, ceil(numel/64) bytes (double-quantized absmax).
+   scales : optional output, ceil(ceil(numel/64)/256) floats, 4-byte aligned; required
+            when codes8 is given, ignored otherwise. */
+typedef struct {
+  const void* w;
+  int64_t numel;
+  int32_t dtype; /* aqnf4_dtype */
+  int32_t reserved; /* must be 0 */
+  uint8_t* packed;
+  float* absmax;
+  uint8_t* codes8;
+  float* scales;
+} aqnf4_layer;
+
+/* Human-readable name of a status code (static string). */
+AQNF4_API const char* aqnf4_status_string(aqnf4_status st);
+
+/* The NF4 codebook ("QLoRA", "How It Works"; "QLoRA Explained", "NF4").  Host only.
+   levels[16]: ascending, levels[0] = -1, levels[7] = 0 exactly, levels[15] = +1.  The 8
+   positive levels are standard-normal quantiles at probabilities spaced evenly from 1/2
+   (excluded) to p_max, the 7 negative ones likewise, all divided by the quantile of p_max;
+   computed in binary64 and rounded to binary32.
+   mids[15]: mids[j] = binary32 rounding of (levels[j] + levels[j+1]) / 2 taken in binary64.
+   p_max <= 0 selects the default 1 - (1/32 + 1/30)/2, which the kernels use.
+   Returns AQNF4_ERR_INVALID_ARG for null pointers or p_max outside (1/2, 1). */
+AQNF4_API aqnf4_status aqnf4_codebook(double p_max, float levels[16], float mids[15]);
+
+/* Blockwise absmax NF4 quantization of one tensor ("QLoRA", "How It Works").
+   w (device, 16-byte aligned): n elements of dtype.  For each 64-element block b:
+     a_b = max |x| (NaN if any element is NaN);
+     v = fl(x * fl(1/a_b)) (a block with a_b below 2^-126 is scaled by 2^64 first; a block
+         with a_b = 0 gets code 7 throughout);
+     code = number of midpoints m_j with v > m_j.
+   packed (device, 16-byte aligned, ceil(n/2) bytes) and absmax (device, 4-byte aligned,
+   ceil(n/64) floats) are outputs; either may be NULL.  dev_flag may be NULL.
+   Errors: INVALID_ARG (w NULL, n < 1), ALIGNMENT, DTYPE, CUDA. */
+AQNF4_API aqnf4_status aqnf4_quantize(const void* w, int32_t dtype, int64_t n, uint8_t* packed,
+                            float* absmax, int32_t* dev_flag, cudaStream_t stream);
+
+/* Double quantization of an absmax array ("QLoRA", "How It Works": quantizing the
+   quantization constants; "QLoRA Explained", "Double Quantization").
+   absmax (device, 4-byte aligned): nb constants.  For each block of 256 constants
+   s = max a (NaN if any is NaN) is stored in scales[d] and each constant becomes
+   code8 = round_half_even(fl(fl(a / s) * 255)); s = 0 gives codes 0; a NaN or infinite s
+   gives codes 0 and sets dev_flag.  Storage per parameter: 8/64 + 32/(64*256) bits instead
+   of 32/64, i.e. 0.373 bits saved.
+   codes8 (device, nb bytes), scales (device, 4-byte aligned, ceil(nb/256) floats).
+   Errors: INVALID_ARG (NULL pointer, nb < 1), ALIGNMENT, CUDA. */
+AQNF4_API aqnf4_status aqnf4_double_quant(const float* absmax, int64_t nb, uint8_t* codes8,
+                                float* scales, int32_t* dev_flag, cudaStream_t stream);
+
+/* NF4 -> 16-bit dequantization ("QLoRA", "How It Works": dequantized to 16 bits on the fly).
+   packed (device, 16-byte aligned): ceil(n/2) bytes.  The block constant is
+   a' = fl(fl(code8/255) * scales[b/256]) when codes8 is non-NULL (then scales is required),
+   else a' = absmax[b].  out[i] = dtype_rn(fl(levels[code_i] * a')).
+   out (device, 16-byte aligned): n elements of out_dtype.
+   Errors: INVALID_ARG (NULL pointers, n < 1), ALIGNMENT, DTYPE, CUDA. */
+AQNF4_API aqnf4_status aqnf4_dequantize(const uint8_t* packed, const uint8_t* codes8,
+                              const float* scales, const float* absmax, int64_t n,
+                              int32_t out_dtype, void* out, cudaStream_t stream);
+
+/* Bytes of device workspace aqnf4_layer_error needs for these layers (host only; 0 when
+   the arguments are invalid). */
+AQNF4_API size_t aqnf4_workspace_size(const aqnf4_layer* layers, int32_t num_layers);
+
+/* The AQLoRA scoring pass (arxivdaily 2608.23816, "English abstract": layers ranked by NF4
+   reconstruction error), fused with NF4 quantization, packing and double quantization.
+   layers: HOST array of num_layers descriptors (device pointers inside).  Each layer is
+   quantized as in aqnf4_quantize; its optional outputs (packed, absmax, codes8 + scales)
+   are written; and, with w_hat = dtype_rn(fl(levels[code] * a_b)),
+     sq_err[l] = sum (x - w_hat)^2,  sq_w[l] = sum x^2,
+     rel_err[l] = sqrt(sq_err[l] / sq_w[l])  (0 when sq_w[l] = 0; NaN after a NaN/inf input).
+   The sums are taken in a fixed order, so repeated calls give identical bits.
+   workspace (device, 256-byte aligned) of at least aqnf4_workspace_size bytes, contents
+   ignored on entry.  sq_err, sq_w (device double[num_layers]) and rel_err (device
+   float[num_layers]) are outputs; any may be NULL.
+   Errors: INVALID_ARG, ALIGNMENT, DTYPE, WORKSPACE, CUDA. */
+AQNF4_API aqnf4_status aqnf4_layer_error(const aqnf4_layer* layers, int32_t num_layers, void* workspace,
+                               size_t ws_bytes, double* sq_err, double* sq_w, float* rel_err,
+                               int32_t* dev_flag, cudaStream_t stream);
+
+/* Top-K under a byte budget (arxivdaily 2608.23816, "English abstract": keep the top-K in
+   fp16 under a memory budget; "AQLoRA: ...", "Technical Details": configurable budget).
+   Layers are ranked by rel_err descending, equal scores by lower index first, NaN scores
+   last.  Walking the ranking, layers are kept until the next one would exceed k_cap layers
+   (k_cap < 0: no cap) or push the summed cost_bytes above budget_bytes.
+   rel_err (device float[L]), cost_bytes (device int64[L]) are inputs; sel_idx (device
+   int32[L]) receives the whole ranking, of which the first *k_out entries are the kept
+   layers; k_out (device int32[1]).  Runs in one thread block, O(L^2 / 1024) time.
+   Errors: INVALID_ARG (NULL pointer, L < 1, budget_bytes < 0), ALIGNMENT, CUDA. */
+AQNF4_API aqnf4_status aqnf4_select_topk(const float* rel_err, const int64_t* cost_bytes, int32_t L,
+                               int64_t budget_bytes, int32_t k_cap, int32_t* sel_idx,
+                               int32_t* k_out, cudaStream_t stream);
+
+/* Incremental bytes of keeping an n-element layer in 16 bits instead of its NF4 storage
+   (packed + codes8 + scales): 2n - (ceil(n/2) + ceil(n/64) + 4*ceil(ceil(n/64)/256)).
+   Host only; -1 for n < 1.  (The 0.2 GiB extra memory of the abstract's quality setting is
+   read as a budget on this quantity.) */
+AQNF4_API int64_t aqnf4_cost_bytes(int64_t n);
+
+/* Number of kernels this library has launched in this process (host counter). */
+AQNF4_API uint64_t aqnf4_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* AQNF4_H */

@@ -1,0 +1,283 @@
+"""Python binding of libaqnf4 (ctypes): argument marshalling only.
+
+Every function named ``aqnf4_*`` here calls the C entry point of the same name; tensors
+are passed by ``data_ptr()``, streams by their CUDA handle.  Every step of the NF4 pass
+runs in the library's CUDA kernels: there is no fallback of any kind, and loading fails
+loudly when the library has not been built (``python -m quantized_lora_setup_b200.build``).
+
+The helpers below the raw bindings (``quantize``, ``score_layers`` ...) only allocate the
+output tensors with torch and then call the bindings.
+"""
+import ctypes
+import os
+from typing import List, Optional, Sequence
+
+import torch
+
+from .build import LIB
+
+AQNF4_OK = 0
+AQNF4_ERR_INVALID_ARG = 1
+AQNF4_ERR_ALIGNMENT = 2
+AQNF4_ERR_DTYPE = 3
+AQNF4_ERR_NONFINITE = 4
+AQNF4_ERR_CUDA = 5
+AQNF4_ERR_TIMEOUT = 6
+AQNF4_ERR_WORKSPACE = 7
+
+AQNF4_F16 = 0
+AQNF4_BF16 = 1
+
+_DT_CODE = {torch.float16: AQNF4_F16, torch.bfloat16: AQNF4_BF16}
+_CODE_DT = {AQNF4_F16: torch.float16, AQNF4_BF16: torch.bfloat16}
+
+BLOCK = 64
+DQ_BLOCK = 256
+
+
+class Aqnf4Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class aqnf4_layer(ctypes.Structure):
+    """Mirror of the C struct aqnf4_layer (see include/aqnf4.h)."""
+
+    _fields_ = [
+        ("w", ctypes.c_void_p),
+        ("numel", ctypes.c_int64),
+        ("dtype", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+        ("packed", ctypes.c_void_p),
+        ("absmax", ctypes.c_void_p),
+        ("codes8", ctypes.c_void_p),
+        ("scales", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def library() -> ctypes.CDLL:
+    """Load libaqnf4.so (raises if it was never built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB):
+        raise ImportError(
+            f"libaqnf4.so is missing ({LIB}); build it with "
+            "`python -m quantized_lora_setup_b200.build`")
+    lib = ctypes.CDLL(LIB)
+    P, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    st = ctypes.c_int
+    lib.aqnf4_status_string.argtypes = [st]
+    lib.aqnf4_status_string.restype = ctypes.c_char_p
+    lib.aqnf4_codebook.argtypes = [ctypes.c_double, P, P]
+    lib.aqnf4_codebook.restype = st
+    lib.aqnf4_quantize.argtypes = [P, i32, i64, P, P, P, P]
+    lib.aqnf4_quantize.restype = st
+    lib.aqnf4_double_quant.argtypes = [P, i64, P, P, P, P]
+    lib.aqnf4_double_quant.restype = st
+    lib.aqnf4_dequantize.argtypes = [P, P, P, P, i64, i32, P, P]
+    lib.aqnf4_dequantize.restype = st
+    lib.aqnf4_workspace_size.argtypes = [P, i32]
+    lib.aqnf4_workspace_size.restype = ctypes.c_size_t
+    lib.aqnf4_layer_error.argtypes = [P, i32, P, ctypes.c_size_t, P, P, P, P, P]
+    lib.aqnf4_layer_error.restype = st
+    lib.aqnf4_select_topk.argtypes = [P, P, i32, i64, i32, P, P, P]
+    lib.aqnf4_select_topk.restype = st
+    lib.aqnf4_cost_bytes.argtypes = [i64]
+    lib.aqnf4_cost_bytes.restype = i64
+    lib.aqnf4_launch_count.argtypes = []
+    lib.aqnf4_launch_count.restype = ctypes.c_uint64
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return library().aqnf4_status_string(status).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != AQNF4_OK:
+        raise Aqnf4Error(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def dtype_code(dtype: torch.dtype) -> int:
+    try:
+        return _DT_CODE[dtype]
+    except KeyError:
+        raise Aqnf4Error(AQNF4_ERR_DTYPE, "dtype") from None
+
+
+# ---------------------------------------------------------------- raw bindings
+
+
+def aqnf4_codebook(p_max: float = 0.0):
+    """(levels float32[16], mids float32[15]) as numpy arrays, from the library."""
+    import numpy as np
+    levels = np.zeros(16, np.float32)
+    mids = np.zeros(15, np.float32)
+    _check(library().aqnf4_codebook(p_max, levels.ctypes.data_as(ctypes.c_void_p),
+                                    mids.ctypes.data_as(ctypes.c_void_p)), "aqnf4_codebook")
+    return levels, mids
+
+
+def aqnf4_quantize(w: torch.Tensor, packed: Optional[torch.Tensor], absmax: Optional[torch.Tensor],
+                   dev_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    _check(library().aqnf4_quantize(_ptr(w), dtype_code(w.dtype), w.numel(), _ptr(packed),
+                                    _ptr(absmax), _ptr(dev_flag), _stream(stream)),
+           "aqnf4_quantize")
+
+
+def aqnf4_double_quant(absmax: torch.Tensor, codes8: torch.Tensor, scales: torch.Tensor,
+                       dev_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    _check(library().aqnf4_double_quant(_ptr(absmax), absmax.numel(), _ptr(codes8), _ptr(scales),
+                                        _ptr(dev_flag), _stream(stream)), "aqnf4_double_quant")
+
+
+def aqnf4_dequantize(packed: torch.Tensor, codes8: Optional[torch.Tensor],
+                     scales: Optional[torch.Tensor], absmax: Optional[torch.Tensor], n: int,
+                     out: torch.Tensor, stream=None) -> None:
+    _check(library().aqnf4_dequantize(_ptr(packed), _ptr(codes8), _ptr(scales), _ptr(absmax), n,
+                                      dtype_code(out.dtype), _ptr(out), _stream(stream)),
+           "aqnf4_dequantize")
+
+
+def make_layers(layers: Sequence[dict]):
+    """ctypes array of aqnf4_layer from dicts with keys w, packed, absmax, codes8, scales."""
+    arr = (aqnf4_layer * len(layers))()
+    for i, d in enumerate(layers):
+        w = d["w"]
+        arr[i].w = w.data_ptr()
+        arr[i].numel = w.numel()
+        arr[i].dtype = dtype_code(w.dtype)
+        arr[i].reserved = 0
+        for key in ("packed", "absmax", "codes8", "scales"):
+            t = d.get(key)
+            setattr(arr[i], key, None if t is None else t.data_ptr())
+    return arr
+
+
+def aqnf4_workspace_size(layers) -> int:
+    arr = layers if isinstance(layers, ctypes.Array) else make_layers(layers)
+    return int(library().aqnf4_workspace_size(arr, len(arr)))
+
+
+def aqnf4_layer_error(layers, workspace: torch.Tensor, sq_err: Optional[torch.Tensor],
+                      sq_w: Optional[torch.Tensor], rel_err: Optional[torch.Tensor],
+                      dev_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    arr = layers if isinstance(layers, ctypes.Array) else make_layers(layers)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(library().aqnf4_layer_error(arr, len(arr), _ptr(workspace), nbytes, _ptr(sq_err),
+                                       _ptr(sq_w), _ptr(rel_err), _ptr(dev_flag),
+                                       _stream(stream)), "aqnf4_layer_error")
+
+
+def aqnf4_select_topk(rel_err: torch.Tensor, cost_bytes: torch.Tensor, budget_bytes: int,
+                      k_cap: int, sel_idx: torch.Tensor, k_out: torch.Tensor,
+                      stream=None) -> None:
+    _check(library().aqnf4_select_topk(_ptr(rel_err), _ptr(cost_bytes), rel_err.numel(),
+                                       int(budget_bytes), int(k_cap), _ptr(sel_idx), _ptr(k_out),
+                                       _stream(stream)), "aqnf4_select_topk")
+
+
+def aqnf4_cost_bytes(n: int) -> int:
+    return int(library().aqnf4_cost_bytes(n))
+
+
+def aqnf4_launch_count() -> int:
+    return int(library().aqnf4_launch_count())
+
+
+# ---------------------------------------------------------------- allocating helpers
+
+
+def nblocks(n: int) -> int:
+    return (n + BLOCK - 1) // BLOCK
+
+
+def nscales(n: int) -> int:
+    return (nblocks(n) + DQ_BLOCK - 1) // DQ_BLOCK
+
+
+def quantize(w: torch.Tensor, stream=None):
+    """NF4-quantize one tensor: returns (packed uint8[ceil(n/2)], absmax float32[ceil(n/64)])."""
+    n = w.numel()
+    packed = torch.empty((n + 1) // 2, dtype=torch.uint8, device=w.device)
+    absmax = torch.empty(nblocks(n), dtype=torch.float32, device=w.device)
+    aqnf4_quantize(w, packed, absmax, None, stream)
+    return packed, absmax
+
+
+def double_quant(absmax: torch.Tensor, stream=None):
+    nb = absmax.numel()
+    codes8 = torch.empty(nb, dtype=torch.uint8, device=absmax.device)
+    scales = torch.empty((nb + DQ_BLOCK - 1) // DQ_BLOCK, dtype=torch.float32, device=absmax.device)
+    aqnf4_double_quant(absmax, codes8, scales, None, stream)
+    return codes8, scales
+
+
+def dequantize(packed: torch.Tensor, n: int, dtype: torch.dtype = torch.bfloat16,
+               codes8=None, scales=None, absmax=None, stream=None) -> torch.Tensor:
+    out = torch.empty(n, dtype=dtype, device=packed.device)
+    aqnf4_dequantize(packed, codes8, scales, absmax, n, out, stream)
+    return out
+
+
+class NF4Storage:
+    """Device buffers of one layer's NF4 storage (packed nibbles + double-quantized absmax)."""
+
+    def __init__(self, n: int, device, with_absmax: bool = False):
+        self.n = n
+        self.packed = torch.empty((n + 1) // 2, dtype=torch.uint8, device=device)
+        self.codes8 = torch.empty(nblocks(n), dtype=torch.uint8, device=device)
+        self.scales = torch.empty(nscales(n), dtype=torch.float32, device=device)
+        self.absmax = (torch.empty(nblocks(n), dtype=torch.float32, device=device)
+                       if with_absmax else None)
+
+
+def score_layers(weights: List[torch.Tensor], storages: Optional[List[NF4Storage]] = None,
+                 stream=None):
+    """Run the fused quantize+score pass: returns (sq_err f64[L], sq_w f64[L], rel_err f32[L])."""
+    dev = weights[0].device
+    L = len(weights)
+    descs = []
+    for i, w in enumerate(weights):
+        d = {"w": w}
+        if storages is not None:
+            s = storages[i]
+            d.update(packed=s.packed, codes8=s.codes8, scales=s.scales, absmax=s.absmax)
+        descs.append(d)
+    arr = make_layers(descs)
+    ws = torch.empty(max(aqnf4_workspace_size(arr), 256), dtype=torch.uint8, device=dev)
+    sq_err = torch.empty(L, dtype=torch.float64, device=dev)
+    sq_w = torch.empty(L, dtype=torch.float64, device=dev)
+    rel = torch.empty(L, dtype=torch.float32, device=dev)
+    aqnf4_layer_error(arr, ws, sq_err, sq_w, rel, None, stream)
+    return sq_err, sq_w, rel
+
+
+def select_topk(rel_err: torch.Tensor, cost_bytes: torch.Tensor, budget_bytes: int,
+                k_cap: int = -1, stream=None):
+    """Returns (ranking int32[L] on the device, k int32[1] on the device)."""
+    L = rel_err.numel()
+    sel = torch.empty(L, dtype=torch.int32, device=rel_err.device)
+    k = torch.empty(1, dtype=torch.int32, device=rel_err.device)
+    aqnf4_select_topk(rel_err, cost_bytes, budget_bytes, k_cap, sel, k, stream)
+    return sel, k

@@ -1,0 +1,125 @@
+// dequant.cu -- NF4 -> 16-bit dequantization (aqnf4_dequantize).
+//
+// "QLoRA", "How It Works": the 4-bit weights are dequantized to 16 bits on the fly for the
+// forward and backward pass.  For element i of block b = i / 64:
+//   a' = fl(fl(code8[b] / 255) * scales[b / 256])   (double-quantized constants), or
+//   a' = absmax[b]                                  (plain constants);
+//   out[i] = dtype_rn(fl(level[code_i] * a')).
+//
+// HBM-bound (0.516 B/element in, 2 B/element out).  A lane handles chunks of 8 elements:
+// one 4-byte load of packed codes, one 16-byte store.  The 32 lanes of a warp take 32
+// consecutive chunks, so loads and stores are fully coalesced; a warp-iteration covers
+// 8 x 32 chunks for memory-level parallelism.  The level lookup is a warp shuffle whose
+// source lane is the nibble itself (lanes 16..31 mirror 0..15, so the shifted word needs
+// no mask).  fl(c / 255) for the 256 possible bytes is tabulated in shared memory with a
+// correctly rounded divide.
+#include "device.cuh"
+
+namespace aqnf4 {
+namespace {
+
+constexpr int kChunksPerLane = 8;
+
+struct DqParams {
+  float level[16];
+};
+
+template <int DT>
+__global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ packed,
+                                                 const uint8_t* __restrict__ codes8,
+                                                 const float* __restrict__ scales,
+                                                 const float* __restrict__ absmax, int64_t n,
+                                                 uint16_t* __restrict__ out,
+                                                 const __grid_constant__ DqParams p) {
+  using F = Fmt<DT>;
+  __shared__ float frac[256];
+  const int t = threadIdx.x, lane = t & 31;
+  frac[t] = __fdiv_rn(static_cast<float>(t), 255.0f);
+  __syncthreads();
+  const float tab_level = p.level[lane & 15];
+
+  const int64_t nchunk = (n + 7) >> 3;
+  const int64_t full_chunks = n >> 3;
+  const int64_t warp_id = (static_cast<int64_t>(blockIdx.x) * blockDim.x + t) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  constexpr int64_t kGroup = 32 * kChunksPerLane;
+
+  for (int64_t g = warp_id; g * kGroup < nchunk; g += nwarps) {
+    uint32_t wd[kChunksPerLane];
+    float ap[kChunksPerLane];
+#pragma unroll
+    for (int j = 0; j < kChunksPerLane; ++j) {
+      const int64_t c = g * kGroup + j * 32 + lane;
+      wd[j] = 0;
+      ap[j] = 0.0f;
+      if (c < full_chunks) {
+        wd[j] = __ldg(reinterpret_cast<const uint32_t*>(packed) + c);
+      } else if (c < nchunk) {  // last, partial chunk: read only the bytes that exist
+        const int64_t nbytes = (n + 1) >> 1;
+        for (int64_t byte = c * 4; byte < nbytes; ++byte)
+          wd[j] |= static_cast<uint32_t>(packed[byte]) << (8 * (byte - c * 4));
+      }
+      if (c < nchunk) {
+        const int64_t b = c >> 3;  // 8 chunks per 64-element block
+        ap[j] = codes8 ? __fmul_rn(frac[__ldg(codes8 + b)], __ldg(scales + (b >> 8)))
+                       : __ldg(absmax + b);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kChunksPerLane; ++j) {
+      const uint32_t w = wd[j];
+      const float2 a2 = make_float2(ap[j], ap[j]);
+      uint32_t o[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        // byte h holds element 2h in its high nibble and element 2h+1 in its low nibble
+        const float q0 = __shfl_sync(kFull, tab_level, static_cast<int>(w >> (8 * h + 4)));
+        const float q1 = __shfl_sync(kFull, tab_level, static_cast<int>(w >> (8 * h)));
+        const float2 v = mul2_rn(make_float2(q0, q1), a2);
+        o[h] = F::pack_rn(v.x, v.y);
+      }
+      const int64_t c = g * kGroup + j * 32 + lane;
+      if (c < full_chunks) {
+        *reinterpret_cast<uint4*>(out + 8 * c) = make_uint4(o[0], o[1], o[2], o[3]);
+      } else if (c < nchunk) {
+        for (int e = 0; e < 8 && 8 * c + e < n; ++e)
+          out[8 * c + e] = static_cast<uint16_t>(o[e >> 1] >> ((e & 1) * 16));
+      }
+    }
+  }
+}
+
+}  // namespace
+}  // namespace aqnf4
+
+using namespace aqnf4;
+
+extern "C" aqnf4_status aqnf4_dequantize(const uint8_t* packed, const uint8_t* codes8,
+                                         const float* scales, const float* absmax, int64_t n,
+                                         int32_t out_dtype, void* out, cudaStream_t stream) {
+  if (!packed || !out || n < 1) return AQNF4_ERR_INVALID_ARG;
+  if (codes8 ? !scales : !absmax) return AQNF4_ERR_INVALID_ARG;
+  if (!valid_dtype(out_dtype)) return AQNF4_ERR_DTYPE;
+  if (!is_aligned(packed, 16) || !is_aligned(out, 16) || !is_aligned(scales, 4) ||
+      !is_aligned(absmax, 4))
+    return AQNF4_ERR_ALIGNMENT;
+  const Tables* tb = default_tables();
+  if (!tb) return AQNF4_ERR_CUDA;
+  DqParams p;
+  for (int i = 0; i < 16; ++i) p.level[i] = tb->level[i];
+  const int64_t nchunk = (n + 7) >> 3;
+  const int64_t groups = (nchunk + 32 * kChunksPerLane - 1) / (32 * kChunksPerLane);
+  const int sms = current_sm_count();
+  int64_t grid = static_cast<int64_t>(sms > 0 ? sms : 1) * 8;  // 8 warps per CTA
+  const int64_t need = (groups + 7) / 8;
+  if (grid > need) grid = need;
+  uint16_t* o = static_cast<uint16_t*>(out);
+  if (out_dtype == AQNF4_BF16)
+    k_dequant<AQNF4_BF16><<<static_cast<unsigned>(grid), 256, 0, stream>>>(packed, codes8, scales,
+                                                                           absmax, n, o, p);
+  else
+    k_dequant<AQNF4_F16><<<static_cast<unsigned>(grid), 256, 0, stream>>>(packed, codes8, scales,
+                                                                          absmax, n, o, p);
+  count_launches(1);
+  return cudaGetLastError() == cudaSuccess ? AQNF4_OK : AQNF4_ERR_CUDA;
+}

@@ -1,0 +1,147 @@
+"""The C-ABI library on the host (no GPU): it loads, exports every declared symbol, its
+host-only functions agree with the oracle, and argument checks fail before any launch."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from quantized_lora_setup_b200 import aqnf4
+from quantized_lora_setup_b200.build import INCLUDE, build
+
+HEADER = os.path.join(INCLUDE, "aqnf4.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return aqnf4.library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"AQNF4_API\s+[\w\s\*]+?\b(aqnf4_\w+)\s*\(", text)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    for required in ("aqnf4_codebook", "aqnf4_quantize", "aqnf4_double_quant",
+                     "aqnf4_dequantize", "aqnf4_layer_error", "aqnf4_select_topk",
+                     "aqnf4_workspace_size", "aqnf4_cost_bytes"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 10
+    for name in names:
+        assert hasattr(lib, name), name
+
+
+def test_library_codebook_matches_oracle_bit_for_bit(lib):
+    lv, md = aqnf4.aqnf4_codebook()
+    olv, omd = oracle.codebook()
+    assert np.array_equal(lv.view(np.uint32), olv.view(np.uint32))
+    assert np.array_equal(md.view(np.uint32), omd.view(np.uint32))
+    for pm in (0.9, 0.99, 0.75):
+        lv, md = aqnf4.aqnf4_codebook(pm)
+        olv, omd = oracle.codebook(pm)
+        assert np.array_equal(lv, olv) and np.array_equal(md, omd)
+    with pytest.raises(aqnf4.Aqnf4Error):
+        aqnf4.aqnf4_codebook(1.5)
+
+
+def test_cost_bytes_matches_oracle(lib):
+    for n in (1, 2, 63, 64, 65, 16383, 16384, 16385, 4096 * 11008, 5120 * 13824):
+        assert aqnf4.aqnf4_cost_bytes(n) == oracle.cost_bytes(n)
+    assert aqnf4.aqnf4_cost_bytes(0) == -1
+
+
+class FakeTensor:
+    """Just enough of a tensor for the binding's marshalling (never dereferenced)."""
+
+    def __init__(self, addr, numel, dtype=None, itemsize=1):
+        self._addr, self._numel, self.dtype, self._itemsize = addr, numel, dtype, itemsize
+
+    def data_ptr(self):
+        return self._addr
+
+    def numel(self):
+        return self._numel
+
+    def element_size(self):
+        return self._itemsize
+
+
+def layer(addr=0x10000, numel=100, dtype=aqnf4.AQNF4_BF16, **kw):
+    d = aqnf4.aqnf4_layer()
+    d.w, d.numel, d.dtype, d.reserved = addr, numel, dtype, kw.get("reserved", 0)
+    d.packed = kw.get("packed")
+    d.absmax = kw.get("absmax")
+    d.codes8 = kw.get("codes8")
+    d.scales = kw.get("scales")
+    return d
+
+
+def test_workspace_size(lib):
+    arr = (aqnf4.aqnf4_layer * 3)(layer(numel=1), layer(numel=16384), layer(numel=16385))
+    assert lib.aqnf4_workspace_size(arr, 3) == 256  # 4 tiles x 16 B, rounded up to 256
+    big = (aqnf4.aqnf4_layer * 1)(layer(numel=16384 * 100))
+    assert lib.aqnf4_workspace_size(big, 1) == 1792
+    assert lib.aqnf4_workspace_size(arr, 0) == 0
+    assert lib.aqnf4_workspace_size(None, 3) == 0
+
+
+def test_argument_checks_return_before_any_launch(lib):
+    V = ctypes.c_void_p
+    before = lib.aqnf4_launch_count()
+    # quantize
+    assert lib.aqnf4_quantize(None, 1, 100, V(0x10000), V(0x20000), None, None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert lib.aqnf4_quantize(V(0x10000), 1, 0, None, None, None, None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert lib.aqnf4_quantize(V(0x10000), 7, 10, None, None, None, None) == aqnf4.AQNF4_ERR_DTYPE
+    assert lib.aqnf4_quantize(V(0x10008), 1, 10, None, None, None, None) == aqnf4.AQNF4_ERR_ALIGNMENT
+    assert lib.aqnf4_quantize(V(0x10000), 1, 10, V(0x20004), None, None, None) == aqnf4.AQNF4_ERR_ALIGNMENT
+    # double quant
+    assert lib.aqnf4_double_quant(None, 10, V(0x100), V(0x200), None, None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert lib.aqnf4_double_quant(V(0x102), 10, V(0x100), V(0x200), None, None) == aqnf4.AQNF4_ERR_ALIGNMENT
+    # dequantize: codes8 requires scales, plain needs absmax
+    assert lib.aqnf4_dequantize(V(0x100), V(0x200), None, None, 10, 1, V(0x300), None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert lib.aqnf4_dequantize(V(0x100), None, None, None, 10, 1, V(0x300), None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert lib.aqnf4_dequantize(V(0x100), None, None, V(0x400), 10, 5, V(0x300), None) == aqnf4.AQNF4_ERR_DTYPE
+    assert lib.aqnf4_dequantize(V(0x100), None, None, V(0x400), 10, 1, V(0x308), None) == aqnf4.AQNF4_ERR_ALIGNMENT
+    # layer error
+    one = (aqnf4.aqnf4_layer * 1)(layer())
+    ws = V(0x100000)
+    assert lib.aqnf4_layer_error(one, 0, ws, 4096, None, None, None, None, None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    bad = (aqnf4.aqnf4_layer * 1)(layer(reserved=1))
+    assert lib.aqnf4_layer_error(bad, 1, ws, 4096, None, None, None, None, None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    bad = (aqnf4.aqnf4_layer * 1)(layer(codes8=0x5000))
+    assert lib.aqnf4_layer_error(bad, 1, ws, 4096, None, None, None, None, None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    bad = (aqnf4.aqnf4_layer * 1)(layer(dtype=9))
+    assert lib.aqnf4_layer_error(bad, 1, ws, 4096, None, None, None, None, None) == aqnf4.AQNF4_ERR_DTYPE
+    bad = (aqnf4.aqnf4_layer * 1)(layer(addr=0x10002))
+    assert lib.aqnf4_layer_error(bad, 1, ws, 4096, None, None, None, None, None) == aqnf4.AQNF4_ERR_ALIGNMENT
+    assert lib.aqnf4_layer_error(one, 1, None, 4096, None, None, None, None, None) == aqnf4.AQNF4_ERR_WORKSPACE
+    assert lib.aqnf4_layer_error(one, 1, V(0x100010), 4096, None, None, None, None, None) == aqnf4.AQNF4_ERR_WORKSPACE
+    assert lib.aqnf4_layer_error(one, 1, ws, 8, None, None, None, None, None) == aqnf4.AQNF4_ERR_WORKSPACE
+    assert lib.aqnf4_layer_error(one, 1, ws, 4096, V(0x104), None, None, None, None) == aqnf4.AQNF4_ERR_ALIGNMENT
+    # select
+    assert lib.aqnf4_select_topk(V(0x100), V(0x200), 5, -1, -1, V(0x300), V(0x400), None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert lib.aqnf4_select_topk(V(0x100), V(0x200), 0, 10, -1, V(0x300), V(0x400), None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert lib.aqnf4_select_topk(V(0x100), V(0x204), 5, 10, -1, V(0x300), V(0x400), None) == aqnf4.AQNF4_ERR_ALIGNMENT
+    assert lib.aqnf4_launch_count() == before
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        assert aqnf4.status_string(code)
+    assert aqnf4.status_string(99) == "unknown status"
+
+
+def test_binding_names_match_the_header():
+    for name in declared_functions():
+        if name in ("aqnf4_status_string",):
+            continue
+        assert callable(getattr(aqnf4, name)), name

@@ -1,0 +1,277 @@
+"""GPU parity: every libaqnf4 entry point against the CPU oracle on the same seeded bytes.
+
+Bit-exact: NF4 codes / packed bytes, absmax, DQ bytes and scales, dequantized values,
+the selected layer set.  Floating point: per-layer sq_err, sq_w and rel_err within a
+relative 1e-5.  That bound follows from the kernel's arithmetic: each thread sums at most
+64 squares in binary32 (relative error <= 64 u, u = 2^-24), a warp adds 32 such partial
+sums in binary32 (<= 5 u more) and everything above that is binary64, so the relative
+error of a sum of non-negative terms stays below 70 u ~ 4.2e-6; the square root halves it
+for rel_err.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_lora_setup_b200 import aqnf4, synth
+
+pytestmark = pytest.mark.gpu
+RTOL = 1e-5
+
+DT = {torch.float16: oracle.F16, torch.bfloat16: oracle.BF16}
+
+
+def bits(t):
+    return synth.bits_u16(t)
+
+
+def u32(a):
+    return np.ascontiguousarray(a, np.float32).view(np.uint32)
+
+
+def same_float_bits(got, ref):
+    g, r = np.asarray(got, np.float32), np.asarray(ref, np.float32)
+    return np.all((u32(g) == u32(r)) | (np.isnan(g) & np.isnan(r)))
+
+
+SIZES = [1, 2, 3, 7, 8, 9, 15, 16, 17, 63, 64, 65, 127, 128, 1000, 16383, 16384, 16385,
+         3 * 16384 + 17, 100003, 262145]
+
+
+@pytest.mark.parametrize("dt", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("n", SIZES)
+def test_quantize_ragged_sizes(cuda, dt, n):
+    w = synth.random_bits_host(n, seed=n, dtype=dt)
+    packed, absmax = aqnf4.quantize(w.to(cuda))
+    op, oa, _ = oracle.quantize(bits(w), DT[dt])
+    assert np.array_equal(packed.cpu().numpy(), op)
+    assert same_float_bits(absmax.cpu().numpy(), oa)
+
+
+def _all_values_blocks(dt, a):
+    """Every finite value of dt with |x| <= a, 63 per block, each block led by +a."""
+    allb = torch.arange(65536, dtype=torch.int32).to(torch.int16).view(dt)
+    v = allb.float()
+    keep = torch.isfinite(v) & (v.abs() <= a)
+    vals = allb[keep]
+    nblk = (vals.numel() + 62) // 63
+    pad = torch.zeros(nblk * 63 - vals.numel(), dtype=dt)
+    body = torch.cat([vals, pad]).reshape(nblk, 63)
+    lead = torch.full((nblk, 1), a, dtype=torch.float32).to(dt)
+    return torch.cat([lead, body], dim=1).reshape(-1)
+
+
+@pytest.mark.parametrize("dt,a", [
+    (torch.bfloat16, 1.0), (torch.bfloat16, 0.02), (torch.bfloat16, 3.0e38),
+    (torch.bfloat16, 1e-30), (torch.bfloat16, 2.0 ** -128), (torch.bfloat16, 2.0 ** -126),
+    (torch.float16, 1.0), (torch.float16, 65504.0), (torch.float16, 1e-3), (torch.float16, 3e-7)])
+def test_quantize_every_value_of_the_format(cuda, dt, a):
+    """All 16-bit values against one block maximum: covers every midpoint neighbourhood."""
+    w = _all_values_blocks(dt, a)
+    packed, absmax = aqnf4.quantize(w.to(cuda))
+    op, oa, _ = oracle.quantize(bits(w), DT[dt])
+    assert np.array_equal(packed.cpu().numpy(), op)
+    assert same_float_bits(absmax.cpu().numpy(), oa)
+    se, sw, rel = aqnf4.score_layers([w.to(cuda)])
+    ose, osw, orel = oracle.layer_error(bits(w), DT[dt])
+    assert se.item() == pytest.approx(ose, rel=RTOL)
+    assert sw.item() == pytest.approx(osw, rel=RTOL)
+    assert rel.item() == pytest.approx(orel, rel=RTOL)
+
+
+def test_quantize_special_blocks(cuda):
+    rng = np.random.default_rng(0)
+    blocks = []
+    blocks.append(np.zeros(64))                       # zero block -> code 7
+    blocks.append(-np.zeros(64))                      # negative zeros
+    z = np.zeros(64); z[17] = -0.5; blocks.append(z)  # single value, negative maximum
+    blocks.append(rng.standard_normal(64) * 1e-39)    # subnormal absmax (bf16)
+    blocks.append(-np.abs(rng.standard_normal(64)))   # all negative
+    blocks.append(np.full(64, 0.25))                  # constant block
+    blocks.append(rng.standard_normal(64) * 5e37)     # near the top of the range
+    w = torch.from_numpy(np.concatenate(blocks).astype(np.float32)).to(torch.bfloat16)
+    packed, absmax = aqnf4.quantize(w.to(cuda))
+    op, oa, _ = oracle.quantize(bits(w), oracle.BF16)
+    assert np.array_equal(packed.cpu().numpy(), op)
+    assert same_float_bits(absmax.cpu().numpy(), oa)
+
+
+@pytest.mark.parametrize("dt", [torch.float16, torch.bfloat16])
+def test_nonfinite_input_sets_the_flag(cuda, dt):
+    w = synth.random_bits_host(64 * 40, seed=3, dtype=dt)
+    w[5] = float("nan")
+    w[64 * 7 + 3] = float("inf")
+    w[64 * 9] = float("-inf")
+    flag = torch.zeros(1, dtype=torch.int32, device=cuda)
+    n = w.numel()
+    packed = torch.empty((n + 1) // 2, dtype=torch.uint8, device=cuda)
+    absmax = torch.empty(aqnf4.nblocks(n), dtype=torch.float32, device=cuda)
+    aqnf4.aqnf4_quantize(w.to(cuda), packed, absmax, flag)
+    assert flag.item() == aqnf4.AQNF4_ERR_NONFINITE
+    op, oa, onf = oracle.quantize(bits(w), DT[dt])
+    assert onf
+    assert np.array_equal(packed.cpu().numpy(), op)
+    assert same_float_bits(absmax.cpu().numpy(), oa)
+    flag.zero_()
+    clean = synth.random_bits_host(64 * 40, seed=4, dtype=dt)
+    rel = torch.empty(2, device=cuda)
+    aqnf4.aqnf4_layer_error([{"w": clean.to(cuda)}, {"w": w.to(cuda)}],
+                            torch.empty(4096, dtype=torch.uint8, device=cuda), None, None, rel,
+                            flag)
+    assert flag.item() == aqnf4.AQNF4_ERR_NONFINITE
+    assert math.isnan(rel[1].item()) and not math.isnan(rel[0].item())
+
+
+def _run_layers(cuda, weights, with_absmax=True):
+    stor = [aqnf4.NF4Storage(w.numel(), cuda, with_absmax=with_absmax) for w in weights]
+    se, sw, rel = aqnf4.score_layers([w.to(cuda) for w in weights], stor)
+    torch.cuda.synchronize()
+    return stor, se.cpu().numpy(), sw.cpu().numpy(), rel.cpu().numpy()
+
+
+def _check_layer(w, st, se, sw, rel):
+    dt = DT[w.dtype]
+    b = bits(w)
+    op, oa, _ = oracle.quantize(b, dt)
+    oc, osc, _ = oracle.double_quant(oa)
+    ose, osw, orel = oracle.layer_error(b, dt)
+    assert np.array_equal(st.packed.cpu().numpy(), op)
+    if st.absmax is not None:
+        assert same_float_bits(st.absmax.cpu().numpy(), oa)
+    assert np.array_equal(st.codes8.cpu().numpy(), oc)
+    assert same_float_bits(st.scales.cpu().numpy(), osc)
+    assert se == pytest.approx(ose, rel=RTOL, abs=0)
+    assert sw == pytest.approx(osw, rel=RTOL, abs=0)
+    assert rel == pytest.approx(orel, rel=RTOL, abs=0)
+    return orel
+
+
+def _selection_agrees(gpu_rel, ora_rel, cost, budget, k_cap, gpu_sel):
+    """Selected set bit-exact; near-ties at the cut are checked on the oracle's scores."""
+    ref = oracle.select_topk(ora_rel, cost, budget, k_cap)
+    if sorted(gpu_sel) == sorted(ref):
+        return True
+    # tie-ambiguous only if the GPU scores at the cut are within 2e-5 of each other
+    order = oracle.select_topk(gpu_rel, cost, 1 << 62, -1)
+    k = len(gpu_sel)
+    if 0 < k < len(order):
+        a, b = gpu_rel[order[k - 1]], gpu_rel[order[k]]
+        if abs(a - b) <= 2e-5 * max(abs(a), abs(b)):
+            return True
+    return False
+
+
+def test_tiny_model_end_to_end(cuda):
+    wl = synth.tiny(0)
+    weights = [synth.layer_host(s, wl.seed, i) for i, s in enumerate(wl.layers)]
+    stor, se, sw, rel = _run_layers(cuda, weights)
+    orel = [_check_layer(w, st, se[i], sw[i], rel[i]) for i, (w, st) in enumerate(zip(weights, stor))]
+    cost = np.array([aqnf4.aqnf4_cost_bytes(s.numel) for s in wl.layers], np.int64)
+    sel, k = aqnf4.select_topk(torch.from_numpy(rel).to(cuda), torch.from_numpy(cost).to(cuda),
+                               wl.budgets[0], wl.k_cap)
+    kk = k.item()
+    got = sel.cpu().numpy()[:kk].tolist()
+    assert kk == 2
+    assert got == oracle.select_topk(rel, cost, wl.budgets[0], wl.k_cap)
+    assert _selection_agrees(rel, orel, cost, wl.budgets[0], wl.k_cap, got)
+    assert sorted(got) == sorted(i for i, s in enumerate(wl.layers) if s.dist == "t")
+
+
+def test_mixed_dtypes_ragged_layers(cuda):
+    sizes = [1, 65, 16383, 16385, 50000, 7, 100003, 64, 32768 + 1]
+    weights = [synth.random_bits_host(n, seed=100 + i,
+                                      dtype=torch.float16 if i % 3 == 0 else torch.bfloat16)
+               for i, n in enumerate(sizes)]
+    weights[4] = weights[4] * 0  # an all-zero layer: rel_err 0
+    stor, se, sw, rel = _run_layers(cuda, weights)
+    for i, (w, st) in enumerate(zip(weights, stor)):
+        _check_layer(w, st, se[i], sw[i], rel[i])
+    assert rel[4] == 0.0
+
+
+def test_more_layers_than_one_launch_holds(cuda):
+    weights = [synth.random_bits_host(64 * (1 + i % 5) + i % 3, seed=i, dtype=torch.bfloat16)
+               for i in range(400)]
+    stor, se, sw, rel = _run_layers(cuda, weights, with_absmax=False)
+    for i in (0, 1, 383, 384, 385, 399):
+        _check_layer(weights[i], stor[i], se[i], sw[i], rel[i])
+
+
+def test_repeat_calls_are_bit_identical(cuda):
+    wl = synth.tiny(1)
+    weights = [synth.layer_host(s, wl.seed, i) for i, s in enumerate(wl.layers)]
+    a = _run_layers(cuda, weights)
+    b = _run_layers(cuda, weights)
+    for x, y in zip(a[1:], b[1:]):
+        assert np.array_equal(x.view(np.uint8), y.view(np.uint8))
+    for s1, s2 in zip(a[0], b[0]):
+        assert torch.equal(s1.packed, s2.packed) and torch.equal(s1.codes8, s2.codes8)
+
+
+def test_double_quant_standalone_and_fused_agree(cuda):
+    rng = np.random.default_rng(5)
+    for nb in (1, 255, 256, 257, 1000, 4096 + 3):
+        a = np.abs(rng.standard_normal(nb)).astype(np.float32) * 0.03
+        if nb > 300:
+            a[256:512] = 0.0  # a zero DQ block
+        codes8, scales = aqnf4.double_quant(torch.from_numpy(a).to(cuda))
+        oc, osc, _ = oracle.double_quant(a)
+        assert np.array_equal(codes8.cpu().numpy(), oc)
+        assert same_float_bits(scales.cpu().numpy(), osc)
+    # the fused pass's DQ equals the standalone one on its own absmax
+    w = synth.random_bits_host(16384 * 3 + 999, seed=9, dtype=torch.bfloat16).to(cuda)
+    st = aqnf4.NF4Storage(w.numel(), cuda, with_absmax=True)
+    aqnf4.score_layers([w], [st])
+    c2, s2 = aqnf4.double_quant(st.absmax)
+    assert torch.equal(c2, st.codes8) and torch.equal(s2, st.scales)
+
+
+def test_double_quant_nonfinite_flag(cuda):
+    a = np.ones(600, np.float32)
+    a[300] = np.nan
+    flag = torch.zeros(1, dtype=torch.int32, device=cuda)
+    codes8 = torch.empty(600, dtype=torch.uint8, device=cuda)
+    scales = torch.empty(3, dtype=torch.float32, device=cuda)
+    aqnf4.aqnf4_double_quant(torch.from_numpy(a).to(cuda), codes8, scales, flag)
+    assert flag.item() == aqnf4.AQNF4_ERR_NONFINITE
+    oc, osc, _ = oracle.double_quant(a)
+    assert np.array_equal(codes8.cpu().numpy(), oc)
+    assert same_float_bits(scales.cpu().numpy(), osc)
+
+
+@pytest.mark.parametrize("out_dt", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("n", [1, 2, 7, 8, 9, 63, 64, 65, 1023, 16384 + 3, 200001])
+def test_dequantize_matches_oracle(cuda, out_dt, n):
+    w = synth.random_bits_host(n, seed=n + 7, dtype=torch.bfloat16)
+    op, oa, _ = oracle.quantize(bits(w), oracle.BF16)
+    oc, osc, _ = oracle.double_quant(oa)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(cuda)
+    got = aqnf4.dequantize(dev(op), n, out_dt, codes8=dev(oc), scales=dev(osc))
+    ref = oracle.dequantize(op, n, DT[out_dt], codes8=oc, scales=osc)
+    assert np.array_equal(bits(got.cpu()), ref)
+    got2 = aqnf4.dequantize(dev(op), n, out_dt, absmax=dev(oa))
+    ref2 = oracle.dequantize(op, n, DT[out_dt], absmax=oa)
+    assert np.array_equal(bits(got2.cpu()), ref2)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_select_topk_matches_oracle(cuda, seed):
+    rng = np.random.default_rng(seed)
+    L = int(rng.choice([1, 2, 5, 28, 280, 1100, 2500]))
+    e = rng.uniform(0, 1, L).astype(np.float32)
+    e[rng.uniform(size=L) < 0.2] = 0.5  # ties
+    e[rng.uniform(size=L) < 0.05] = np.nan
+    cost = rng.integers(1, 1 << 30, L).astype(np.int64)
+    if seed % 3 == 0:
+        cost[rng.integers(0, L)] = -5  # a layer cheaper in 16 bits than in NF4
+    budget = int(rng.integers(0, int(cost[cost > 0].sum()) + 1))
+    k_cap = int(rng.choice([-1, 0, 1, 3, L]))
+    sel, k = aqnf4.select_topk(torch.from_numpy(e).to(cuda), torch.from_numpy(cost).to(cuda),
+                               budget, k_cap)
+    ref = oracle.select_topk(e, cost, budget, k_cap)
+    got = sel.cpu().numpy()
+    assert got[: k.item()].tolist() == ref
+    full = oracle.select_topk(e, np.zeros(L, np.int64), 0, -1)
+    assert got.tolist() == full  # the whole ranking is returned
