@@ -42,6 +42,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dequant", action="store_true")
+    ap.add_argument("--max-layers", type=int, default=0,
+                    help="use only the first N layers (small cases for profiling)")
     return ap.parse_args()
 
 
@@ -249,6 +251,9 @@ def run_native(args):
     aqnf4.library()
 
     wl = synth.workload(args.workload)
+    if args.max_layers > 0:
+        wl = synth.Workload(wl.name + f"[:{args.max_layers}]", wl.layers[: args.max_layers],
+                            wl.budgets, wl.k_cap, wl.seed)
     L = len(wl.layers)
     parts = lpt_partition([s.numel for s in wl.layers], world)
     mine = parts[rank]

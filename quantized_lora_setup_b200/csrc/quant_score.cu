@@ -9,19 +9,22 @@
 //   per 256 blocks: s = max a_b, code8_b = rint(fl(fl(a_b / s) * 255));
 //   per layer: sum (x - w_hat)^2 and sum x^2 with w_hat = dtype_rn(fl(level[code] * a_b)).
 //
-// The sums are taken per block in the normalised domain, sum ((x - w_hat) r)^2 and
-// sum v^2 in binary32 (each term <= 1, so nothing overflows or underflows for any finite
-// input), then scaled by a_b^2 and summed in binary64 in a fixed order.
+// Each thread sums its block's (x - w_hat)^2 and x^2 in binary32 -- directly when
+// 2^-40 <= a_b <= 2^40, where no term can overflow or underflow; otherwise in the
+// normalised domain ((x - w_hat) r)^2 and v^2, scaled back by a_b^2 -- and the 256 block
+// sums of a tile are added in binary64 in a fixed order.
 //
 // Work decomposition (B200): a tile is 16384 consecutive elements of one layer (one DQ
 // block).  A persistent CTA of 256 threads walks tiles with a grid stride; one thread owns
-// one 64-element block.  A 1-D bulk copy (TMA engine) streams each 32 KB tile into a
-// 2-stage shared-memory ring (two CTAs per SM), so the only global-load instructions are
-// the copies issued by one thread.  Each thread reads its own 128 bytes back with conflict-free 16-byte loads
-// (chunk order rotated per thread), takes the absmax with packed bf16x2/f16x2 max, one
-// correctly rounded reciprocal, and finds each code with one round-toward-minus-infinity
-// FMA (bucket index) plus two warp-shuffle table lookups and one compare.  Packed codes are
-// staged in shared memory and written out with coalesced 16-byte stores.
+// one 64-element block.  A 1-D bulk copy (TMA engine) brings each 32 KB tile into shared
+// memory; three CTAs share an SM, so one CTA's copy overlaps the others' arithmetic.  Each
+// thread reads its own 128 bytes twice with conflict-free 16-byte loads (chunk order
+// rotated per thread): once for the absmax (packed bf16x2/f16x2 max), once to code.  A code
+// costs one round-toward-minus-infinity FMA (bucket index), two warp-shuffle table lookups
+// and one compare; arithmetic on pairs uses Blackwell's packed f32x2 instructions, and
+// w_hat - x comes from the packed 16-bit w_hat with one mixed-precision subtract.  Packed codes are staged in shared memory and leave with coalesced
+// 16-byte stores.  The per-tile extra work (the next bulk copy, the binary64 reduction)
+// rotates over the warps so no warp is always last at the barrier.
 #include <cfloat>
 
 #include "device.cuh"
@@ -30,9 +33,18 @@ namespace aqnf4 {
 namespace {
 
 constexpr int kThreads = 256;  // = kDqBlock: one thread per NF4 block of a tile
-constexpr int kStages = 2;
-constexpr int kMaxLayersPerLaunch = 384;
 constexpr int kWarps = kThreads / 32;
+constexpr int kCtasPerSm = 3;  // 80 registers per thread; 4 spills, 2 leaves latency exposed
+constexpr int kMaxLayersPerLaunch = 384;
+
+// shared memory layout (bytes): one input stage, two packed-output stages, two copies of the
+// per-thread (err, w^2, absmax) floats, two copies of the per-warp absmax, the mbarrier.
+constexpr size_t kOutOff = kTileBytes;
+constexpr size_t kRedOff = kOutOff + 2 * kPackedTileBytes;
+constexpr size_t kRedBytes = 3 * 2 * kThreads * sizeof(float);
+constexpr size_t kMaxOff = kRedOff + kRedBytes;
+constexpr size_t kBarOff = kMaxOff + 2 * kWarps * sizeof(float);
+constexpr size_t kSmemBytes = kBarOff + 16;
 
 struct LayerRec {
   const void* w;
@@ -69,12 +81,6 @@ struct FParams {
   int32_t tile_begin[kMaxLayersPerLaunch + 1];
 };
 
-constexpr size_t kStageBytes = static_cast<size_t>(kStages) * kTileBytes;
-constexpr size_t kOutBytes = 2 * kPackedTileBytes;
-// per tile: one (sum err, sum w^2) double pair per thread and one absmax per warp, twice
-constexpr size_t kRedBytes = 2 * (kThreads * sizeof(double2) + kWarps * sizeof(float));
-constexpr size_t kSmemBytes = kStageBytes + kOutBytes + kRedBytes + kStages * 8 + 16;
-
 __device__ __forceinline__ int find_layer(const QParams& p, int64_t tile) {
   int lo = 0, hi = p.num_layers - 1;  // tile_begin[lo] <= tile < tile_begin[hi + 1]
   while (lo < hi) {
@@ -105,26 +111,26 @@ __device__ __forceinline__ TileGeom tile_geom(const QParams& p, int64_t tile, in
   return g;
 }
 
-// Thread 0: start the bulk copy of `tile` into stage `s`.  A short last tile copies its
-// 16-byte-aligned prefix; the remaining < 8 elements are read from global memory later.
-__device__ __forceinline__ void issue_tile(const QParams& p, int64_t tile, int s, uint8_t* stage,
-                                          uint64_t* bars, uint64_t policy, int& cursor) {
+// Start the bulk copy of `tile` into the stage.  A short last tile copies its
+// 16-byte-aligned prefix; its remaining < 8 elements are read from global memory later.
+__device__ __forceinline__ void issue_tile(const QParams& p, int64_t tile, uint8_t* stage,
+                                          uint32_t bar, uint64_t policy, int& cursor) {
   const TileGeom g = tile_geom(p, tile, cursor);
   const uint32_t bytes = static_cast<uint32_t>(g.cnt * 2) & ~15u;
-  const uint32_t bar = smem_addr(bars + s);
   mbar_arrive_expect_tx(bar, bytes);
   if (bytes) {
     const uint8_t* src = static_cast<const uint8_t*>(p.layers[g.layer].w) + g.tin * kTileBytes;
-    bulk_load(smem_addr(stage + static_cast<size_t>(s) * kTileBytes), src, bytes, bar, policy);
+    bulk_load(smem_addr(stage), src, bytes, bar, policy);
   }
 }
 
 // Generic per-element path for a block whose absmax is 0, below the binary32 normal range,
-// or not finite.  Recomputes this thread's packed words and error sums.
+// or not finite.  Re-reads the block (natural element order) from shared memory, rewrites
+// this thread's packed words and returns the normalised sums (err, w^2) -- scaled by a^2
+// later like the fast path's.
 template <int DT, bool SCORE>
-__device__ __noinline__ void block_generic(const uint32_t* wl, int rot, float a,
-                                           const QParams& p, uint8_t* ost, int t, double* se_out,
-                                           double* sw_out) {
+__device__ __noinline__ float2 block_generic(const uint8_t* my, float a, const QParams& p,
+                                             uint8_t* ost) {
   using F = Fmt<DT>;
   const bool zero = (a == 0.0f);
   const bool finite = (a <= FLT_MAX);
@@ -134,13 +140,13 @@ __device__ __noinline__ void block_generic(const uint32_t* wl, int rot, float a,
     as = __fmul_rn(a, scale);
   }
   const float r = zero ? 0.0f : __frcp_rn(as);
+  const uint16_t* x16 = reinterpret_cast<const uint16_t*>(my);
   float se = 0.0f, sw = 0.0f;
   for (int c = 0; c < 8; ++c) {
-    const int k2 = (c - rot) & 7;
     uint32_t pk = 0;
     for (int i = 0; i < 8; ++i) {
-      const uint32_t wd = wl[4 * k2 + (i >> 1)];
-      const float x = (i & 1) ? F::hi(wd) : F::lo(wd);
+      const uint32_t h = x16[8 * c + i];
+      const float x = F::lo(h);
       int code = 7;
       float v = 0.0f;
       if (!zero) {
@@ -156,32 +162,26 @@ __device__ __noinline__ void block_generic(const uint32_t* wl, int rot, float a,
         sw = __fmaf_rn(v, v, sw);
       }
     }
-    *reinterpret_cast<uint32_t*>(ost + t * 32 + c * 4) = pk;
+    *reinterpret_cast<uint32_t*>(ost + c * 4) = pk;
   }
-  // back to the weights' scale: (a * scale)^2 / scale^2
-  const double as2 = static_cast<double>(as) * static_cast<double>(as);
-  const double inv_s2 = 1.0 / (static_cast<double>(scale) * static_cast<double>(scale));
-  double E = static_cast<double>(se) * as2 * inv_s2;
-  double W = static_cast<double>(sw) * as2 * inv_s2;
-  if (zero) E = W = 0.0;
   if (!finite) {
-    E = W = __longlong_as_double(0x7ff8000000000000ll);
+    se = sw = __int_as_float(0x7fffffff);
     if (p.flag) *p.flag = AQNF4_ERR_NONFINITE;
   }
-  *se_out = E;
-  *sw_out = W;
+  return make_float2(se, sw);
 }
 
 template <int DT, bool SCORE>
-__global__ void __launch_bounds__(kThreads, 2) k_quant_score(const __grid_constant__ QParams p) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_quant_score(const __grid_constant__ QParams p) {
   using F = Fmt<DT>;
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* stage = smem;
-  uint8_t* out_stage = smem + kStageBytes;
-  double2* red_sum = reinterpret_cast<double2*>(out_stage + kOutBytes);        // [2][256]
-  float* red_max = reinterpret_cast<float*>(red_sum + 2 * kThreads);           // [2][8]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStageBytes + kOutBytes + kRedBytes);
-  int* abort_flag = reinterpret_cast<int*>(bars + kStages);
+  float* red = reinterpret_cast<float*>(smem + kRedOff);   // [3 = err, w2, a][2][256]
+  float* wmax = reinterpret_cast<float*>(smem + kMaxOff);  // [2][8]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kBarOff);
+  int* abort_flag = reinterpret_cast<int*>(smem + kBarOff + 8);
+  const uint32_t bar_a = smem_addr(bar);
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   // this lane's entries of the shuffle lookup tables
@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_quant_score(const __grid_consta
   const float tab_level = p.level[lane & 15];
 
   if (t == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(smem_addr(bars + s), 1);
+    mbar_init(bar_a, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -198,145 +198,126 @@ __global__ void __launch_bounds__(kThreads, 2) k_quant_score(const __grid_consta
 
   const int64_t T = p.num_tiles;
   const int64_t stride = gridDim.x;
-  uint64_t policy = 0;
-  int issue_cursor = 0, cursor = 0;
-  if (t == 0) {
-    policy = l2_evict_first_policy();
-    for (int s = 0; s < kStages; ++s) {
-      const int64_t tile = blockIdx.x + s * stride;
-      if (tile < T) issue_tile(p, tile, s, stage, bars, policy, issue_cursor);
-    }
-  }
+  const uint64_t policy = l2_evict_first_policy();
+  int cursor = 0, issue_cursor = 0;
+  if (t == 0 && blockIdx.x < T) issue_tile(p, blockIdx.x, stage, bar_a, policy, issue_cursor);
 
+  const int rot = (t + (t >> 3)) & 7;  // conflict-free 16-byte reads and 4-byte writes
+  const uint8_t* my = stage + t * 128;
   int64_t k = 0;
   bool aborted = false;
   for (int64_t tile = blockIdx.x; tile < T; tile += stride, ++k) {
-    const int s = static_cast<int>(k % kStages);
-    const uint32_t parity = static_cast<uint32_t>((k / kStages) & 1);
-    if (!mbar_wait_bounded(smem_addr(bars + s), parity)) {
+    const int buf = static_cast<int>(k & 1);
+    if (!mbar_wait_bounded(bar_a, static_cast<uint32_t>(buf))) {
       *abort_flag = 1;
       if (p.flag) *p.flag = AQNF4_ERR_TIMEOUT;
     }
-
     const TileGeom g = tile_geom(p, tile, cursor);
     const LayerRec& L = p.layers[g.layer];
     const int nblk = (g.cnt + kBlock - 1) / kBlock;
-    const uint8_t* st = stage + static_cast<size_t>(s) * kTileBytes;
-
-    // ---- this thread's 64 elements into registers
-    uint32_t words[32];
-    int rot;
-    if (g.cnt == kTile) {
-      rot = (t + (t >> 3)) & 7;  // conflict-free for the 16-byte reads and 4-byte writes
-#pragma unroll
-      for (int k2 = 0; k2 < 8; ++k2) {
-        const int c = (k2 + rot) & 7;
-        const uint4 v = *reinterpret_cast<const uint4*>(st + t * 128 + c * 16);
-        words[4 * k2 + 0] = v.x;
-        words[4 * k2 + 1] = v.y;
-        words[4 * k2 + 2] = v.z;
-        words[4 * k2 + 3] = v.w;
-      }
-    } else {
-      rot = 0;
+    if (g.cnt < kTile) {
+      // a layer's short last tile: finish it in shared memory (tail from global, then zeros)
       const int pre = static_cast<int>((static_cast<uint32_t>(g.cnt * 2) & ~15u) >> 1);
+      uint16_t* s16 = reinterpret_cast<uint16_t*>(stage);
       const uint16_t* gw = static_cast<const uint16_t*>(L.w) + g.tin * kTile;
-      const uint16_t* sw = reinterpret_cast<const uint16_t*>(st);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int e = t * 64 + 2 * j;
-        const uint32_t lo = e < g.cnt ? (e < pre ? sw[e] : gw[e]) : 0u;
-        const uint32_t hi = e + 1 < g.cnt ? (e + 1 < pre ? sw[e + 1] : gw[e + 1]) : 0u;
-        words[j] = lo | (hi << 16);
-      }
+      for (int e = pre + t; e < kTile; e += kThreads) s16[e] = e < g.cnt ? gw[e] : 0;
+      fence_proxy_async_smem();
+      __syncthreads();
     }
 
-    // ---- block absmax (NaN propagates)
-    uint32_t m16[16];
+    // ---- pass 1: block absmax (NaN propagates)
+    uint32_t m0 = 0, m1 = 0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) m16[i] = F::absmax2(words[2 * i], words[2 * i + 1]);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) m16[i] = F::absmax2(m16[2 * i], m16[2 * i + 1]);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) m16[i] = F::absmax2(m16[2 * i], m16[2 * i + 1]);
-    m16[0] = F::absmax2(m16[0], m16[1]);
-    m16[1] = F::absmax2(m16[2], m16[3]);
-    m16[0] = F::absmax2(m16[0], m16[1]);
-    m16[0] = F::absmax2(m16[0], __byte_perm(m16[0], 0, 0x1032));
-    const float a = F::abs_lo(m16[0]);
+    for (int k2 = 0; k2 < 8; ++k2) {
+      const uint4 v = lds128(my + ((k2 + rot) & 7) * 16);
+      m0 = F::absmax2(m0, F::absmax2(v.x, v.y));
+      m1 = F::absmax2(m1, F::absmax2(v.z, v.w));
+    }
+    m0 = F::absmax2(m0, m1);
+    m0 = F::absmax2(m0, __byte_perm(m0, 0, 0x1032));
+    const float a = F::abs_lo(m0);
     const bool fast = (a >= 0x1p-126f) && (a <= FLT_MAX);
     const float r = fast ? __frcp_rn(a) : 0.0f;
 
-    // ---- codes, packing, error (all lanes run this so the shuffles stay converged)
-    uint8_t* ost = out_stage + (k & 1) * kPackedTileBytes;
-    float2 err2 = make_float2(0.0f, 0.0f), sw2 = make_float2(0.0f, 0.0f);
+    // ---- pass 2: codes, packing, error (all lanes run this so the shuffles stay converged)
+    // Blocks with 2^-40 <= a <= 2^40 sum (w_hat - x)^2 and x^2 directly in binary32 (no
+    // term can overflow or flush there); the rest take the generic path, which normalises.
+    uint8_t* ost = smem + kOutOff + buf * kPackedTileBytes + t * 32;
+    float2 es2 = make_float2(0.0f, 0.0f), ws2 = make_float2(0.0f, 0.0f);
+    const bool fast_sum = (a >= 0x1p-40f) && (a <= 0x1p40f);
     const float2 r2 = make_float2(r, r), a2 = make_float2(a, a);
     const float2 scale2 = make_float2(15.5f, 15.5f), off2 = make_float2(8388624.0f, 8388624.0f);
 #pragma unroll
     for (int k2 = 0; k2 < 8; ++k2) {
       const int c = (k2 + rot) & 7;
+      const uint4 v4 = lds128(my + c * 16);
+      const uint32_t w4[4] = {v4.x, v4.y, v4.z, v4.w};
       uint32_t pk = 0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint32_t wd = words[4 * k2 + j];
+        const uint32_t wd = w4[j];
         const float2 x = make_float2(F::lo(wd), F::hi(wd));
         const float2 v = mul2_rn(x, r2);
         // floor(15.5 v + 16) lands in the low 5 bits of tt (2^23 <= tt < 2^23 + 32)
         const float2 tt = fma2_rm(v, scale2, off2);
         const int i0 = __float_as_int(tt.x), i1 = __float_as_int(tt.y);
-        const float m0 = __shfl_sync(kFull, tab_mid, i0);
-        const float m1 = __shfl_sync(kFull, tab_mid, i1);
-        const uint32_t c0 = __shfl_sync(kFull, tab_code, i0) + (v.x > m0 ? 1u : 0u);
-        const uint32_t c1 = __shfl_sync(kFull, tab_code, i1) + (v.y > m1 ? 1u : 0u);
+        const float m0s = __shfl_sync(kFull, tab_mid, i0);
+        const float m1s = __shfl_sync(kFull, tab_mid, i1);
+        const uint32_t c0 = __shfl_sync(kFull, tab_code, i0) + (v.x > m0s ? 1u : 0u);
+        const uint32_t c1 = __shfl_sync(kFull, tab_code, i1) + (v.y > m1s ? 1u : 0u);
         pk |= ((c0 << 4) | c1) << (8 * j);
         if (SCORE) {
           const float q0 = __shfl_sync(kFull, tab_level, static_cast<int>(c0));
           const float q1 = __shfl_sync(kFull, tab_level, static_cast<int>(c1));
           const float2 wq = mul2_rn(make_float2(q0, q1), a2);
           const uint32_t hb = F::pack_rn(wq.x, wq.y);
-          const float2 d = mul2_rn(sub2_rn(x, make_float2(F::lo(hb), F::hi(hb))), r2);
-          err2 = fma2_rn(d, d, err2);
-          sw2 = fma2_rn(v, v, sw2);
+          // w_hat - x straight from the packed 16-bit result (the sign does not matter)
+          const float2 d = make_float2(F::sub_lo(hb, x.x), F::sub_hi(hb, x.y));
+          es2 = fma2_rn(d, d, es2);
+          ws2 = fma2_rn(x, x, ws2);
         }
       }
-      *reinterpret_cast<uint32_t*>(ost + t * 32 + c * 4) = pk;
+      *reinterpret_cast<uint32_t*>(ost + c * 4) = pk;
     }
-    const double a2d = static_cast<double>(a) * static_cast<double>(a);
-    double e_t = static_cast<double>(err2.x + err2.y) * a2d;
-    double w_t = static_cast<double>(sw2.x + sw2.y) * a2d;
-    if (!fast) {
-      uint32_t wl[32];  // stack copy: keeps `words` itself in registers
-#pragma unroll
-      for (int j = 0; j < 32; ++j) wl[j] = words[j];
-      block_generic<DT, SCORE>(wl, rot, a, p, ost, t, &e_t, &w_t);
+    float2 sums = make_float2(es2.x + es2.y, ws2.x + ws2.y);
+    // factor that turns this block's sums into weight units once squared
+    float sum_scale = 1.0f;
+    if (!fast || !fast_sum) {
+      sums = block_generic<DT, SCORE>(my, a, p, ost);
+      sum_scale = a;
     }
 
     // ---- tile reductions: DQ scale (max a over the tile's blocks) and error sums
-    float am = t < nblk ? a : 0.0f;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) am = fmax_nan(am, __shfl_xor_sync(kFull, am, off));
-    double2* rs = red_sum + (k & 1) * kThreads;
-    float* rm = red_max + (k & 1) * kWarps;
-    if (SCORE) rs[t] = make_double2(e_t, w_t);
-    if (lane == 0) rm[warp] = am;
+    // a >= 0 or NaN: as unsigned integers the binary32 patterns order like the values, with
+    // every NaN above +inf, so an integer max is the NaN-propagating float max
+    const uint32_t am =
+        __reduce_max_sync(kFull, t < nblk ? __float_as_uint(a) : 0u);
+    float* r_err = red + buf * kThreads;
+    float* r_w2 = red + (2 + buf) * kThreads;
+    float* r_a = red + (4 + buf) * kThreads;
+    if (SCORE) {
+      r_err[t] = sums.x;
+      r_w2[t] = sums.y;
+      r_a[t] = sum_scale;
+    }
+    if (lane == 0) wmax[buf * kWarps + warp] = __uint_as_float(am);
     __syncthreads();
     if (*abort_flag) {
       aborted = true;
       break;
     }
-    if (t == 0) {
-      const int64_t next = tile + kStages * stride;
-      if (next < T) {
-        fence_proxy_async_smem();
-        issue_tile(p, next, s, stage, bars, policy, issue_cursor);
-      }
+    const int lead = static_cast<int>(k & (kWarps - 1));  // warp doing this tile's extra work
+    if (warp == lead && lane == 0 && tile + stride < T) {
+      fence_proxy_async_smem();
+      issue_tile(p, tile + stride, stage, bar_a, policy, issue_cursor);
     }
 
     // ---- outputs
+    const uint4 wa = *reinterpret_cast<const uint4*>(wmax + buf * kWarps);
+    const uint4 wb = *reinterpret_cast<const uint4*>(wmax + buf * kWarps + 4);
+    const float sdq = __uint_as_float(max(max(max(wa.x, wa.y), max(wa.z, wa.w)),
+                                          max(max(wb.x, wb.y), max(wb.z, wb.w))));
     const int64_t blk0 = g.tin * kDqBlock;
-    float sdq = rm[0];
-#pragma unroll
-    for (int w = 1; w < kWarps; ++w) sdq = fmax_nan(sdq, rm[w]);
     if (t < nblk) {
       if (L.absmax) L.absmax[blk0 + t] = a;
       if (L.codes8) L.codes8[blk0 + t] = dq_code(a, sdq);
@@ -345,13 +326,14 @@ __global__ void __launch_bounds__(kThreads, 2) k_quant_score(const __grid_consta
       L.scales[g.tin] = sdq;
       if (!(sdq <= FLT_MAX) && p.flag) *p.flag = AQNF4_ERR_NONFINITE;
     }
-    if (SCORE && warp == 0) {
+    if (SCORE && warp == lead) {
       double se = 0.0, sw = 0.0;
 #pragma unroll
-      for (int j = 0; j < kThreads / 32; ++j) {
-        const double2 v = rs[lane + 32 * j];
-        se += v.x;
-        sw += v.y;
+      for (int j = 0; j < kWarps; ++j) {
+        const int i = lane + 32 * j;
+        const double aa = static_cast<double>(r_a[i]) * static_cast<double>(r_a[i]);
+        se += static_cast<double>(r_err[i]) * aa;
+        sw += static_cast<double>(r_w2[i]) * aa;
       }
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) {
@@ -361,15 +343,16 @@ __global__ void __launch_bounds__(kThreads, 2) k_quant_score(const __grid_consta
       if (lane == 0) p.partials[p.tile_base + tile] = make_double2(se, sw);
     }
     if (L.packed) {
+      const uint8_t* os = smem + kOutOff + buf * kPackedTileBytes;
       uint8_t* gp = L.packed + g.tin * kPackedTileBytes;
       if (g.cnt == kTile) {
 #pragma unroll
         for (int i = t; i < kPackedTileBytes / 16; i += kThreads)
-          *reinterpret_cast<uint4*>(gp + 16 * i) = *reinterpret_cast<const uint4*>(ost + 16 * i);
+          *reinterpret_cast<uint4*>(gp + 16 * i) = lds128(os + 16 * i);
       } else {
         const int nbytes = (g.cnt + 1) >> 1;
         for (int i = t; i < nbytes; i += kThreads) {
-          uint8_t b = ost[i];
+          uint8_t b = os[i];
           if ((g.cnt & 1) && i == nbytes - 1) b &= 0xF0;  // odd length: low nibble stays 0
           gp[i] = b;
         }
@@ -378,12 +361,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_quant_score(const __grid_consta
   }
 
   if (aborted && t == 0) {
-    // let every bulk copy this CTA still has in flight land before the CTA exits
-    for (int64_t kk = k; kk < k + kStages; ++kk) {
-      const int64_t tile = blockIdx.x + kk * stride;
-      if (tile >= T) break;
-      mbar_wait_bounded(smem_addr(bars + (kk % kStages)), static_cast<uint32_t>((kk / kStages) & 1));
-    }
+    // let the bulk copy that timed out land before the CTA (and its shared memory) goes away
+    mbar_wait_bounded(bar_a, static_cast<uint32_t>(k & 1));
   }
 }
 
