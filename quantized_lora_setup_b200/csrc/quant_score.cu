@@ -15,16 +15,18 @@
 // sums of a tile are added in binary64 in a fixed order.
 //
 // Work decomposition (B200): a tile is 16384 consecutive elements of one layer (one DQ
-// block).  A persistent CTA of 256 threads walks tiles with a grid stride; one thread owns
-// one 64-element block.  A 1-D bulk copy (TMA engine) brings each 32 KB tile into shared
-// memory; three CTAs share an SM, so one CTA's copy overlaps the others' arithmetic.  Each
-// thread reads its own 128 bytes twice with conflict-free 16-byte loads (chunk order
-// rotated per thread): once for the absmax (packed bf16x2/f16x2 max), once to code.  A code
-// costs one round-toward-minus-infinity FMA (bucket index), two warp-shuffle table lookups
-// and one compare; arithmetic on pairs uses Blackwell's packed f32x2 instructions, and
-// w_hat - x comes from the packed 16-bit w_hat with one mixed-precision subtract.  Packed codes are staged in shared memory and leave with coalesced
-// 16-byte stores.  The per-tile extra work (the next bulk copy, the binary64 reduction)
-// rotates over the warps so no warp is always last at the barrier.
+// block, 256 NF4 blocks).  A persistent CTA of 128 threads walks tiles with a grid stride;
+// thread t owns NF4 blocks t and t + 128.  A 1-D bulk copy (TMA engine) brings each 32 KB
+// tile into shared memory; four CTAs share an SM, so one CTA's copy overlaps the others'
+// arithmetic.  Each thread reads its blocks twice with conflict-free 16-byte loads (chunk
+// order rotated per thread): once for the absmax (packed bf16x2/f16x2 max), once to code,
+// the two blocks' work interleaved.  A code costs one round-toward-minus-infinity FMA
+// (bucket index), two warp-shuffle table lookups and one compare mask; two codes form a
+// packed byte directly, and the byte indexes the level shuffles.  Arithmetic on pairs uses
+// Blackwell's packed f32x2 instructions, and w_hat - x comes from the packed 16-bit w_hat
+// with one mixed-precision subtract.  Packed codes are staged in shared memory and leave with
+// coalesced 16-byte stores.  The per-tile extra work (the next bulk copy, the binary64
+// reduction) rotates over the warps so no warp is always last at the barrier.
 #include <cfloat>
 
 #include "device.cuh"
@@ -32,16 +34,19 @@
 namespace aqnf4 {
 namespace {
 
-constexpr int kThreads = 256;  // = kDqBlock: one thread per NF4 block of a tile
+// Two NF4 blocks per thread (t and t + 128): their dependency chains interleave, which the
+// shuffle latency needs, and per-tile costs are shared by 128 elements.
+constexpr int kBpt = 2;
+constexpr int kThreads = kDqBlock / kBpt;  // a CTA covers one tile (= one DQ block)
 constexpr int kWarps = kThreads / 32;
-constexpr int kCtasPerSm = 3;  // 80 registers per thread; 4 spills, 2 leaves latency exposed
+constexpr int kCtasPerSm = 4;  // 54 KB of shared memory and 128 registers per thread
 constexpr int kMaxLayersPerLaunch = 384;
 
 // shared memory layout (bytes): one input stage, two packed-output stages, two copies of the
-// per-thread (err, w^2, absmax) floats, two copies of the per-warp absmax, the mbarrier.
+// per-block (err, w^2, scale) floats, two copies of the per-warp absmax, the mbarrier.
 constexpr size_t kOutOff = kTileBytes;
 constexpr size_t kRedOff = kOutOff + 2 * kPackedTileBytes;
-constexpr size_t kRedBytes = 3 * 2 * kThreads * sizeof(float);
+constexpr size_t kRedBytes = 3 * 2 * kDqBlock * sizeof(float);
 constexpr size_t kMaxOff = kRedOff + kRedBytes;
 constexpr size_t kBarOff = kMaxOff + 2 * kWarps * sizeof(float);
 constexpr size_t kSmemBytes = kBarOff + 16;
@@ -130,7 +135,7 @@ __device__ __forceinline__ void issue_tile(const QParams& p, int64_t tile, uint8
 // later like the fast path's.
 template <int DT, bool SCORE>
 __device__ __noinline__ float2 block_generic(const uint8_t* my, float a, const QParams& p,
-                                             uint8_t* ost) {
+                                             uint8_t* ost) {  // ost: this block's 32 bytes
   using F = Fmt<DT>;
   const bool zero = (a == 0.0f);
   const bool finite = (a <= FLT_MAX);
@@ -177,8 +182,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   using F = Fmt<DT>;
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* stage = smem;
-  float* red = reinterpret_cast<float*>(smem + kRedOff);   // [3 = err, w2, a][2][256]
-  float* wmax = reinterpret_cast<float*>(smem + kMaxOff);  // [2][8]
+  float* red = reinterpret_cast<float*>(smem + kRedOff);   // [3 = err, w2, scale][2][256]
+  float* wmax = reinterpret_cast<float*>(smem + kMaxOff);  // [2][kWarps]
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kBarOff);
   int* abort_flag = reinterpret_cast<int*>(smem + kBarOff + 8);
   const uint32_t bar_a = smem_addr(bar);
@@ -187,7 +192,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   // this lane's entries of the shuffle lookup tables
   const float tab_mid = p.bucket_mid[lane];
   const uint32_t tab_code = p.bucket_code[lane];
-  const float tab_level = p.level[lane & 15];
+  const uint32_t tab_code16 = tab_code << 4;  // the same, already in the high nibble
+  const float tab_level = p.level[lane & 15];  // lanes 16..31 mirror 0..15
 
   if (t == 0) {
     mbar_init(bar_a, 1);
@@ -203,7 +209,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   if (t == 0 && blockIdx.x < T) issue_tile(p, blockIdx.x, stage, bar_a, policy, issue_cursor);
 
   const int rot = (t + (t >> 3)) & 7;  // conflict-free 16-byte reads and 4-byte writes
-  const uint8_t* my = stage + t * 128;
   int64_t k = 0;
   bool aborted = false;
   for (int64_t tile = blockIdx.x; tile < T; tile += stride, ++k) {
@@ -225,82 +230,104 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       __syncthreads();
     }
 
-    // ---- pass 1: block absmax (NaN propagates)
-    uint32_t m0 = 0, m1 = 0;
+    // ---- pass 1: absmax of this thread's blocks (NaN propagates)
+    float a[kBpt], r[kBpt];
+    bool fast[kBpt], fast_sum[kBpt];
 #pragma unroll
-    for (int k2 = 0; k2 < 8; ++k2) {
-      const uint4 v = lds128(my + ((k2 + rot) & 7) * 16);
-      m0 = F::absmax2(m0, F::absmax2(v.x, v.y));
-      m1 = F::absmax2(m1, F::absmax2(v.z, v.w));
+    for (int b = 0; b < kBpt; ++b) {
+      const uint8_t* my = stage + (t + b * kThreads) * 128;
+      uint32_t m0 = 0, m1 = 0;
+#pragma unroll
+      for (int k2 = 0; k2 < 8; ++k2) {
+        const uint4 v = lds128(my + ((k2 + rot) & 7) * 16);
+        m0 = F::absmax2(m0, F::absmax2(v.x, v.y));
+        m1 = F::absmax2(m1, F::absmax2(v.z, v.w));
+      }
+      m0 = F::absmax2(m0, m1);
+      m0 = F::absmax2(m0, __byte_perm(m0, 0, 0x1032));
+      a[b] = F::abs_lo(m0);
+      fast[b] = (a[b] >= 0x1p-126f) && (a[b] <= FLT_MAX);
+      // 2^-40 <= a <= 2^40: (w_hat - x)^2 and x^2 cannot overflow or flush in binary32
+      fast_sum[b] = (a[b] >= 0x1p-40f) && (a[b] <= 0x1p40f);
+      r[b] = fast[b] ? __frcp_rn(a[b]) : 0.0f;
     }
-    m0 = F::absmax2(m0, m1);
-    m0 = F::absmax2(m0, __byte_perm(m0, 0, 0x1032));
-    const float a = F::abs_lo(m0);
-    const bool fast = (a >= 0x1p-126f) && (a <= FLT_MAX);
-    const float r = fast ? __frcp_rn(a) : 0.0f;
 
-    // ---- pass 2: codes, packing, error (all lanes run this so the shuffles stay converged)
-    // Blocks with 2^-40 <= a <= 2^40 sum (w_hat - x)^2 and x^2 directly in binary32 (no
-    // term can overflow or flush there); the rest take the generic path, which normalises.
-    uint8_t* ost = smem + kOutOff + buf * kPackedTileBytes + t * 32;
-    float2 es2 = make_float2(0.0f, 0.0f), ws2 = make_float2(0.0f, 0.0f);
-    const bool fast_sum = (a >= 0x1p-40f) && (a <= 0x1p40f);
-    const float2 r2 = make_float2(r, r), a2 = make_float2(a, a);
+    // ---- pass 2: codes, packing, error; the blocks' chains interleave (all lanes run this
+    // so the shuffles stay converged)
+    float2 es2[kBpt], ws2[kBpt];
+#pragma unroll
+    for (int b = 0; b < kBpt; ++b) es2[b] = ws2[b] = make_float2(0.0f, 0.0f);
     const float2 scale2 = make_float2(15.5f, 15.5f), off2 = make_float2(8388624.0f, 8388624.0f);
+    uint8_t* ost = smem + kOutOff + buf * kPackedTileBytes;
 #pragma unroll
     for (int k2 = 0; k2 < 8; ++k2) {
       const int c = (k2 + rot) & 7;
-      const uint4 v4 = lds128(my + c * 16);
-      const uint32_t w4[4] = {v4.x, v4.y, v4.z, v4.w};
-      uint32_t pk = 0;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t wd = w4[j];
-        const float2 x = make_float2(F::lo(wd), F::hi(wd));
-        const float2 v = mul2_rn(x, r2);
-        // floor(15.5 v + 16) lands in the low 5 bits of tt (2^23 <= tt < 2^23 + 32)
-        const float2 tt = fma2_rm(v, scale2, off2);
-        const int i0 = __float_as_int(tt.x), i1 = __float_as_int(tt.y);
-        const float m0s = __shfl_sync(kFull, tab_mid, i0);
-        const float m1s = __shfl_sync(kFull, tab_mid, i1);
-        const uint32_t c0 = __shfl_sync(kFull, tab_code, i0) + (v.x > m0s ? 1u : 0u);
-        const uint32_t c1 = __shfl_sync(kFull, tab_code, i1) + (v.y > m1s ? 1u : 0u);
-        pk |= ((c0 << 4) | c1) << (8 * j);
-        if (SCORE) {
-          const float q0 = __shfl_sync(kFull, tab_level, static_cast<int>(c0));
-          const float q1 = __shfl_sync(kFull, tab_level, static_cast<int>(c1));
-          const float2 wq = mul2_rn(make_float2(q0, q1), a2);
-          const uint32_t hb = F::pack_rn(wq.x, wq.y);
-          // w_hat - x straight from the packed 16-bit result (the sign does not matter)
-          const float2 d = make_float2(F::sub_lo(hb, x.x), F::sub_hi(hb, x.y));
-          es2 = fma2_rn(d, d, es2);
-          ws2 = fma2_rn(x, x, ws2);
+      for (int b = 0; b < kBpt; ++b) {
+        const int blk = t + b * kThreads;
+        const uint4 v4 = lds128(stage + blk * 128 + c * 16);
+        const uint32_t w4[4] = {v4.x, v4.y, v4.z, v4.w};
+        const float2 r2 = make_float2(r[b], r[b]), a2 = make_float2(a[b], a[b]);
+        uint32_t pk = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t wd = w4[j];
+          const float2 x = make_float2(F::lo(wd), F::hi(wd));
+          const float2 v = mul2_rn(x, r2);
+          // floor(15.5 v + 16) lands in the low 5 bits of tt (2^23 <= tt < 2^23 + 32)
+          const float2 tt = fma2_rm(v, scale2, off2);
+          const int i0 = __float_as_int(tt.x), i1 = __float_as_int(tt.y);
+          const float m0s = __shfl_sync(kFull, tab_mid, i0);
+          const float m1s = __shfl_sync(kFull, tab_mid, i1);
+          // byte = code0 << 4 | code1 = (base0 << 4) + base1 + [v0 > m0] * 16 + [v1 > m1]
+          const uint32_t base =
+              __shfl_sync(kFull, tab_code16, i0) + __shfl_sync(kFull, tab_code, i1);
+          const uint32_t byte = base - 16u * static_cast<uint32_t>(gt_mask(v.x, m0s)) -
+                                static_cast<uint32_t>(gt_mask(v.y, m1s));
+          pk = j == 0 ? byte : pk + (byte << (8 * j));
+          if (SCORE) {
+            // the level tables mirror lanes 16..31, so the low 5 bits of byte (code1 and one
+            // bit of code0) and of byte >> 4 (code0) pick the right levels
+            const float q0 = __shfl_sync(kFull, tab_level, static_cast<int>(byte >> 4));
+            const float q1 = __shfl_sync(kFull, tab_level, static_cast<int>(byte));
+            const float2 wq = mul2_rn(make_float2(q0, q1), a2);
+            const uint32_t hb = F::pack_rn(wq.x, wq.y);
+            // w_hat - x straight from the packed 16-bit w_hat (the sign does not matter)
+            const float2 d = make_float2(F::sub_lo(hb, x.x), F::sub_hi(hb, x.y));
+            es2[b] = fma2_rn(d, d, es2[b]);
+            ws2[b] = fma2_rn(x, x, ws2[b]);
+          }
         }
+        *reinterpret_cast<uint32_t*>(ost + blk * 32 + c * 4) = pk;
       }
-      *reinterpret_cast<uint32_t*>(ost + c * 4) = pk;
-    }
-    float2 sums = make_float2(es2.x + es2.y, ws2.x + ws2.y);
-    // factor that turns this block's sums into weight units once squared
-    float sum_scale = 1.0f;
-    if (!fast || !fast_sum) {
-      sums = block_generic<DT, SCORE>(my, a, p, ost);
-      sum_scale = a;
     }
 
-    // ---- tile reductions: DQ scale (max a over the tile's blocks) and error sums
-    // a >= 0 or NaN: as unsigned integers the binary32 patterns order like the values, with
-    // every NaN above +inf, so an integer max is the NaN-propagating float max
-    const uint32_t am =
-        __reduce_max_sync(kFull, t < nblk ? __float_as_uint(a) : 0u);
-    float* r_err = red + buf * kThreads;
-    float* r_w2 = red + (2 + buf) * kThreads;
-    float* r_a = red + (4 + buf) * kThreads;
-    if (SCORE) {
-      r_err[t] = sums.x;
-      r_w2[t] = sums.y;
-      r_a[t] = sum_scale;
+    // ---- per block: sums (generic path where needed) into the reduction buffers
+    float* r_err = red + buf * kDqBlock;
+    float* r_w2 = red + (2 + buf) * kDqBlock;
+    float* r_a = red + (4 + buf) * kDqBlock;
+    uint32_t amax = 0;
+#pragma unroll
+    for (int b = 0; b < kBpt; ++b) {
+      const int blk = t + b * kThreads;
+      float2 sums = make_float2(es2[b].x + es2[b].y, ws2[b].x + ws2[b].y);
+      // factor that turns this block's sums into weight units once squared
+      float sum_scale = 1.0f;
+      if (!fast[b] || !fast_sum[b]) {
+        sums = block_generic<DT, SCORE>(stage + blk * 128, a[b], p, ost + blk * 32);
+        sum_scale = a[b];
+      }
+      if (SCORE) {
+        r_err[blk] = sums.x;
+        r_w2[blk] = sums.y;
+        r_a[blk] = sum_scale;
+      }
+      // a >= 0 or NaN: as unsigned integers the binary32 patterns order like the values,
+      // with every NaN above +inf, so an integer max is the NaN-propagating float max
+      if (blk < nblk) amax = max(amax, __float_as_uint(a[b]));
     }
-    if (lane == 0) wmax[buf * kWarps + warp] = __uint_as_float(am);
+    amax = __reduce_max_sync(kFull, amax);
+    if (lane == 0) wmax[buf * kWarps + warp] = __uint_as_float(amax);
     __syncthreads();
     if (*abort_flag) {
       aborted = true;
@@ -313,14 +340,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
 
     // ---- outputs
-    const uint4 wa = *reinterpret_cast<const uint4*>(wmax + buf * kWarps);
-    const uint4 wb = *reinterpret_cast<const uint4*>(wmax + buf * kWarps + 4);
-    const float sdq = __uint_as_float(max(max(max(wa.x, wa.y), max(wa.z, wa.w)),
-                                          max(max(wb.x, wb.y), max(wb.z, wb.w))));
+    uint32_t sdq_bits = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) sdq_bits = max(sdq_bits, __float_as_uint(wmax[buf * kWarps + w]));
+    const float sdq = __uint_as_float(sdq_bits);
     const int64_t blk0 = g.tin * kDqBlock;
-    if (t < nblk) {
-      if (L.absmax) L.absmax[blk0 + t] = a;
-      if (L.codes8) L.codes8[blk0 + t] = dq_code(a, sdq);
+#pragma unroll
+    for (int b = 0; b < kBpt; ++b) {
+      const int blk = t + b * kThreads;
+      if (blk < nblk) {
+        if (L.absmax) L.absmax[blk0 + blk] = a[b];
+        if (L.codes8) L.codes8[blk0 + blk] = dq_code(a[b], sdq);
+      }
     }
     if (t == 0 && L.codes8) {
       L.scales[g.tin] = sdq;
@@ -329,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (SCORE && warp == lead) {
       double se = 0.0, sw = 0.0;
 #pragma unroll
-      for (int j = 0; j < kWarps; ++j) {
+      for (int j = 0; j < kDqBlock / 32; ++j) {
         const int i = lane + 32 * j;
         const double aa = static_cast<double>(r_a[i]) * static_cast<double>(r_a[i]);
         se += static_cast<double>(r_err[i]) * aa;

@@ -1,0 +1,96 @@
+"""GPU parity at the benchmark's full sizes, in the launch configuration bench.py times.
+
+Every layer of the 1.4B-, 7B- and 14B-shaped models goes through one aqnf4_layer_error
+call (fused quantize + pack + double quantization + error), exactly as in bench.py.  The
+oracle then recomputes a sample of layers one by one (first, middle, last, and one of
+each value distribution): packed codes, DQ bytes and scales must be bit-exact and the
+scores within 1e-5.  The selection at every budget must equal the oracle's selection on
+the same score vector.  The standalone dequantization of a 28672x8192 matrix is checked
+on DQ-block-aligned slices.
+"""
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_lora_setup_b200 import aqnf4, synth
+
+pytestmark = pytest.mark.gpu
+RTOL = 1e-5
+DT = {torch.float16: oracle.F16, torch.bfloat16: oracle.BF16}
+
+
+def _sample(wl):
+    L = len(wl.layers)
+    idx = {0, L // 2, L - 1}
+    seen = set()
+    for i, s in enumerate(wl.layers):
+        if s.dist not in seen:
+            seen.add(s.dist)
+            idx.add(i)
+    return sorted(idx)
+
+
+def _oracle_layer(args):
+    w_host, dt = args
+    b = synth.bits_u16(w_host)
+    op, oa, _ = oracle.quantize(b, dt)
+    oc, osc, _ = oracle.double_quant(oa)
+    ose, osw, orel = oracle.layer_error(b, dt)
+    return op, oc, osc, ose, osw, orel
+
+
+@pytest.mark.parametrize("name", ["1.4b", "7b", "14b"])
+def test_full_model_sampled_layers(cuda, name):
+    wl = synth.workload(name)
+    weights = [synth.layer_device(s, wl.seed, i, cuda) for i, s in enumerate(wl.layers)]
+    stor = [aqnf4.NF4Storage(w.numel(), cuda) for w in weights]
+    se, sw, rel = aqnf4.score_layers(weights, stor)
+    torch.cuda.synchronize()
+    rel_h = rel.cpu().numpy()
+    se_h, sw_h = se.cpu().numpy(), sw.cpu().numpy()
+    assert np.all(np.isfinite(rel_h)) and np.all(rel_h > 0)
+
+    sample = _sample(wl)
+    jobs = [(weights[i].cpu(), DT[wl.layers[i].dtype]) for i in sample]
+    with ThreadPoolExecutor(max_workers=len(jobs)) as ex:
+        results = list(ex.map(_oracle_layer, jobs))
+    for i, (op, oc, osc, ose, osw, orel) in zip(sample, results):
+        assert np.array_equal(stor[i].packed.cpu().numpy(), op), f"packed, layer {i}"
+        assert np.array_equal(stor[i].codes8.cpu().numpy(), oc), f"codes8, layer {i}"
+        assert np.array_equal(stor[i].scales.cpu().numpy().view(np.uint32),
+                              osc.view(np.uint32)), f"scales, layer {i}"
+        assert se_h[i] == pytest.approx(ose, rel=RTOL)
+        assert sw_h[i] == pytest.approx(osw, rel=RTOL)
+        assert rel_h[i] == pytest.approx(orel, rel=RTOL)
+
+    cost = np.array([aqnf4.aqnf4_cost_bytes(s.numel) for s in wl.layers], np.int64)
+    cost_d = torch.from_numpy(cost).to(cuda)
+    for budget in wl.budgets:
+        sel, k = aqnf4.select_topk(rel, cost_d, budget, wl.k_cap)
+        got = sel.cpu().numpy()[: k.item()].tolist()
+        assert got == oracle.select_topk(rel_h, cost, budget, wl.k_cap)
+        assert sum(cost[got]) <= budget
+
+
+def test_full_size_dequantize(cuda):
+    rows, cols = synth.DEQUANT_SHAPES[-1]
+    n = rows * cols
+    w = synth.normal_matrix_device(rows, cols, seed=7, device=cuda)
+    st = aqnf4.NF4Storage(n, cuda)
+    aqnf4.score_layers([w], [st])
+    out = aqnf4.dequantize(st.packed, n, torch.bfloat16, codes8=st.codes8, scales=st.scales)
+    torch.cuda.synchronize()
+    tile = 16384  # one DQ block of weights
+    ntiles = n // tile
+    for t in (0, 1, ntiles // 3, ntiles - 1):
+        e0, e1 = t * tile, (t + 1) * tile
+        ref = oracle.dequantize(st.packed[e0 // 2: e1 // 2].cpu().numpy(), tile, oracle.BF16,
+                                codes8=st.codes8[e0 // 64: e1 // 64].cpu().numpy(),
+                                scales=st.scales[t: t + 1].cpu().numpy())
+        assert np.array_equal(synth.bits_u16(out[e0:e1].cpu()), ref)
+    # the reconstruction stays close to the source: NF4 error of a normal matrix
+    err = (out.float() - w.reshape(-1).float()).square().sum() / w.float().square().sum()
+    assert 0.005 < float(err.sqrt()) < 0.15
