@@ -28,7 +28,8 @@ if ROOT not in sys.path:
 METRIC = "NF4 quantize+score GB/s (fp16 weights read) and % of HBM roofline; dequant GB/s"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SRC = os.path.join(ROOT, "quantized_lora_setup_b200", "csrc", "quant_score.cu")
+KERNEL_SRCS = [os.path.join(ROOT, "quantized_lora_setup_b200", "csrc", f)
+               for f in ("quant_score.cu", "device.cuh")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "k_quant_score_7b.md")
 
 
@@ -89,11 +90,14 @@ def oracle_pass(sample):
 
 
 def build_oracle_sample(wl, threads, per_thread_elems, layer_tensors=None):
-    """One slice per thread: the first elements of the workload's first `threads` layers."""
+    """One equal-size slice per thread: the first elements of the workload's first
+    `threads` layers (equal sizes keep the threads busy for the same time)."""
     from quantized_lora_setup_b200 import synth
     import oracle
     sample = []
-    for i in range(min(threads, len(wl.layers))):
+    nl = min(threads, len(wl.layers))
+    per_thread_elems = min([per_thread_elems] + [wl.layers[i].numel for i in range(nl)])
+    for i in range(nl):
         spec = wl.layers[i]
         if layer_tensors is not None:
             w = layer_tensors[i].reshape(-1)[: min(spec.numel, per_thread_elems)].cpu()
@@ -215,17 +219,22 @@ def measured_hbm_peak():
 
 def recorded_traffic():
     """Per-launch DRAM bytes of k_quant_score from the committed ncu summary, if it was
-    taken on the current kernel source (its sha256 is recorded beside the number)."""
+    taken on the current kernel sources (their sha256 is recorded beside the number)."""
     try:
         text = open(TRAFFIC_FILE).read()
-        src = hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()
+        h = hashlib.sha256()
+        for f in KERNEL_SRCS:
+            with open(f, "rb") as fh:
+                h.update(fh.read())
+        src = h.hexdigest()
     except OSError:
         return None
     vals = {}
     for line in text.splitlines():
-        if ":" in line and line.strip().startswith(("traffic_bytes_per_launch", "source_sha256")):
+        line = line.strip().lstrip("-").strip()
+        if ":" in line and line.startswith(("traffic_bytes_per_launch", "source_sha256")):
             k, v = line.split(":", 1)
-            vals[k.strip().strip("`- ")] = v.strip().strip("` ")
+            vals[k.strip()] = v.strip().strip("` ")
     if vals.get("source_sha256") != src:
         return None
     try:
