@@ -152,6 +152,21 @@ AQNF4_API aqnf4_status aqnf4_layer_error(const aqnf4_layer* layers, int32_t num_
                                size_t ws_bytes, double* sq_err, double* sq_w, float* rel_err,
                                int32_t* dev_flag, cudaStream_t stream);
 
+/* Same as aqnf4_layer_error but without a workspace argument (no counterpart on the
+   pages: this is a calling convenience).  For callers that have no way to provide device
+   memory at the call site -- for example a plugin or C FFI layer that only receives device
+   pointers from its host framework, or code running where the framework forbids new device
+   allocations -- the per-tile partial sums go to a scratch array built into the library
+   (8 MiB per device, held until the process exits).  Limit: the layers may span at most
+   2^19 tiles of 16384 elements (8.6e9 weights); larger requests return AQNF4_ERR_WORKSPACE
+   and should be split.  The first call on a device looks up the scratch address with that
+   device current; make it before any stream capture.  All calls on a device share the
+   scratch, so calls that overlap on the GPU race: serialise them.  The library allocates
+   nothing here either.  Other arguments and errors as for aqnf4_layer_error. */
+AQNF4_API aqnf4_status aqnf4_layer_error_noalloc(const aqnf4_layer* layers, int32_t num_layers,
+                                                 double* sq_err, double* sq_w, float* rel_err,
+                                                 int32_t* dev_flag, cudaStream_t stream);
+
 /* Top-K under a byte budget (arxivdaily 2608.23816, "English abstract": keep the top-K in
    fp16 under a memory budget; "AQLoRA: ...", "Technical Details": configurable budget).
    Layers are ranked by rel_err descending, equal scores by lower index first, NaN scores

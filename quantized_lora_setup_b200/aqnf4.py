@@ -85,6 +85,8 @@ def library() -> ctypes.CDLL:
     lib.aqnf4_workspace_size.restype = ctypes.c_size_t
     lib.aqnf4_layer_error.argtypes = [P, i32, P, ctypes.c_size_t, P, P, P, P, P]
     lib.aqnf4_layer_error.restype = st
+    lib.aqnf4_layer_error_noalloc.argtypes = [P, i32, P, P, P, P, P]
+    lib.aqnf4_layer_error_noalloc.restype = st
     lib.aqnf4_select_topk.argtypes = [P, P, i32, i64, i32, P, P, P]
     lib.aqnf4_select_topk.restype = st
     lib.aqnf4_cost_bytes.argtypes = [i64]
@@ -187,6 +189,16 @@ def aqnf4_layer_error(layers, workspace: torch.Tensor, sq_err: Optional[torch.Te
     _check(library().aqnf4_layer_error(arr, len(arr), _ptr(workspace), nbytes, _ptr(sq_err),
                                        _ptr(sq_w), _ptr(rel_err), _ptr(dev_flag),
                                        _stream(stream)), "aqnf4_layer_error")
+
+
+def aqnf4_layer_error_noalloc(layers, sq_err: Optional[torch.Tensor],
+                              sq_w: Optional[torch.Tensor], rel_err: Optional[torch.Tensor],
+                              dev_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    """aqnf4_layer_error with the library's built-in scratch instead of a workspace."""
+    arr = layers if isinstance(layers, ctypes.Array) else make_layers(layers)
+    _check(library().aqnf4_layer_error_noalloc(arr, len(arr), _ptr(sq_err), _ptr(sq_w),
+                                               _ptr(rel_err), _ptr(dev_flag), _stream(stream)),
+           "aqnf4_layer_error_noalloc")
 
 
 def aqnf4_select_topk(rel_err: torch.Tensor, cost_bytes: torch.Tensor, budget_bytes: int,

@@ -28,6 +28,7 @@
 // coalesced 16-byte stores.  The per-tile extra work (the next bulk copy, the binary64
 // reduction) rotates over the warps so no warp is always last at the barrier.
 #include <cfloat>
+#include <mutex>
 
 #include "device.cuh"
 
@@ -480,9 +481,24 @@ aqnf4_status check_layer(const aqnf4_layer& L) {
 }
 
 }  // namespace
+
+// Built-in scratch for aqnf4_layer_error_noalloc: one (err, w^2) double pair per
+// 16384-element tile, enough for 2^19 tiles (8.6e9 weights) in one call.  Every GPU that
+// loads this library holds these 8 MiB until the process exits.
+constexpr int64_t kNoallocTiles = int64_t(1) << 19;
+static __device__ __align__(256) double2 g_noalloc_scratch[kNoallocTiles];
+
 }  // namespace aqnf4
 
 using namespace aqnf4;
+
+namespace {
+// Device address of g_noalloc_scratch, looked up once per device.  On the host the array's
+// name is only a stand-in for the device copy and must never reach a kernel.
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kMaxDevices] = {};
+}  // namespace
 
 extern "C" {
 
@@ -579,6 +595,38 @@ aqnf4_status aqnf4_layer_error(const aqnf4_layer* layers, int32_t num_layers, vo
     i += n;
   }
   return AQNF4_OK;
+}
+
+// Same pass as aqnf4_layer_error, for callers that cannot hand over device memory: the
+// per-tile partial sums go to the library's own fixed scratch array instead of a workspace.
+// The first call on each device looks the array's device address up (with that device
+// current); make that first call before any stream capture on the device.  Nothing in the
+// array needs clearing between calls: every tile slot a call reads was written earlier in
+// the same call.  All calls on a device share the one array, so calls whose kernels
+// overlap on the GPU (for example on two streams) race and must be serialised by the caller.
+aqnf4_status aqnf4_layer_error_noalloc(const aqnf4_layer* layers, int32_t num_layers,
+                                       double* sq_err, double* sq_w, float* rel_err,
+                                       int32_t* dev_flag, cudaStream_t stream) {
+  if (!layers || num_layers < 1) return AQNF4_ERR_INVALID_ARG;
+  const size_t need = aqnf4_workspace_size(layers, num_layers);
+  if (need == 0) return AQNF4_ERR_INVALID_ARG;
+  const size_t have = sizeof(g_noalloc_scratch);
+  if (need > have) return AQNF4_ERR_WORKSPACE;  // more than 2^19 tiles: split the call
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return AQNF4_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr)
+        return AQNF4_ERR_CUDA;
+      g_noalloc_ptr[dev] = ptr;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  return aqnf4_layer_error(layers, num_layers, scratch, have, sq_err, sq_w, rel_err, dev_flag,
+                           stream);
 }
 
 }  // extern "C"
