@@ -26,7 +26,7 @@
 // Blackwell's packed f32x2 instructions, and w_hat - x comes from the packed 16-bit w_hat
 // with one mixed-precision subtract.  Packed codes are staged in shared memory and leave with
 // coalesced 16-byte stores.  The per-tile extra work (the next bulk copy, the binary64
-// reduction) rotates over the warps so no warp is always last at the barrier.
+// reduction) rotates over the warps so no warp is always last at a barrier.
 #include <cfloat>
 #include <mutex>
 
@@ -40,16 +40,18 @@ namespace {
 constexpr int kBpt = 2;
 constexpr int kThreads = kDqBlock / kBpt;  // a CTA covers one tile (= one DQ block)
 constexpr int kWarps = kThreads / 32;
-constexpr int kCtasPerSm = 4;  // 54 KB of shared memory and 128 registers per thread
+constexpr int kCtasPerSm = 4;  // 44 KB of shared memory and 128 registers per thread, no spills
 constexpr int kMaxLayersPerLaunch = 384;
 
-// shared memory layout (bytes): one input stage, two packed-output stages, two copies of the
-// per-block (err, w^2, scale) floats, two copies of the per-warp absmax, the mbarrier.
+// shared memory layout (bytes): one input stage, the packed-output stage, the per-block
+// (err, w^2, scale) floats, the per-warp absmax, the mbarrier and abort word.  The output
+// and reduction buffers are single: a second barrier at the end of each tile separates
+// their readers from the next tile's writers (double buffers cost registers that spill).
 constexpr size_t kOutOff = kTileBytes;
-constexpr size_t kRedOff = kOutOff + 2 * kPackedTileBytes;
-constexpr size_t kRedBytes = 3 * 2 * kDqBlock * sizeof(float);
+constexpr size_t kRedOff = kOutOff + kPackedTileBytes;
+constexpr size_t kRedBytes = 3 * kDqBlock * sizeof(float);
 constexpr size_t kMaxOff = kRedOff + kRedBytes;
-constexpr size_t kBarOff = kMaxOff + 2 * kWarps * sizeof(float);
+constexpr size_t kBarOff = kMaxOff + 16 * sizeof(float);
 constexpr size_t kSmemBytes = kBarOff + 16;
 
 struct LayerRec {
@@ -183,8 +185,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   using F = Fmt<DT>;
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* stage = smem;
-  float* red = reinterpret_cast<float*>(smem + kRedOff);   // [3 = err, w2, scale][2][256]
-  float* wmax = reinterpret_cast<float*>(smem + kMaxOff);  // [2][kWarps]
+  float* red = reinterpret_cast<float*>(smem + kRedOff);   // [3 = err, w2, scale][256]
+  float* wmax = reinterpret_cast<float*>(smem + kMaxOff);  // [kWarps]
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kBarOff);
   int* abort_flag = reinterpret_cast<int*>(smem + kBarOff + 8);
   const uint32_t bar_a = smem_addr(bar);
@@ -213,8 +215,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   int64_t k = 0;
   bool aborted = false;
   for (int64_t tile = blockIdx.x; tile < T; tile += stride, ++k) {
-    const int buf = static_cast<int>(k & 1);
-    if (!mbar_wait_bounded(bar_a, static_cast<uint32_t>(buf))) {
+    if (!mbar_wait_bounded(bar_a, static_cast<uint32_t>(k & 1))) {
       *abort_flag = 1;
       if (p.flag) *p.flag = AQNF4_ERR_TIMEOUT;
     }
@@ -259,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
     for (int b = 0; b < kBpt; ++b) es2[b] = ws2[b] = make_float2(0.0f, 0.0f);
     const float2 scale2 = make_float2(15.5f, 15.5f), off2 = make_float2(8388624.0f, 8388624.0f);
-    uint8_t* ost = smem + kOutOff + buf * kPackedTileBytes;
+    uint8_t* ost = smem + kOutOff;
 #pragma unroll
     for (int k2 = 0; k2 < 8; ++k2) {
       const int c = (k2 + rot) & 7;
@@ -304,9 +305,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
 
     // ---- per block: sums (generic path where needed) into the reduction buffers
-    float* r_err = red + buf * kDqBlock;
-    float* r_w2 = red + (2 + buf) * kDqBlock;
-    float* r_a = red + (4 + buf) * kDqBlock;
+    float* r_err = red;
+    float* r_w2 = red + kDqBlock;
+    float* r_a = red + 2 * kDqBlock;
     uint32_t amax = 0;
 #pragma unroll
     for (int b = 0; b < kBpt; ++b) {
@@ -328,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       if (blk < nblk) amax = max(amax, __float_as_uint(a[b]));
     }
     amax = __reduce_max_sync(kFull, amax);
-    if (lane == 0) wmax[buf * kWarps + warp] = __uint_as_float(amax);
+    if (lane == 0) wmax[warp] = __uint_as_float(amax);
     __syncthreads();
     if (*abort_flag) {
       aborted = true;
@@ -343,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     // ---- outputs
     uint32_t sdq_bits = 0;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) sdq_bits = max(sdq_bits, __float_as_uint(wmax[buf * kWarps + w]));
+    for (int w = 0; w < kWarps; ++w) sdq_bits = max(sdq_bits, __float_as_uint(wmax[w]));
     const float sdq = __uint_as_float(sdq_bits);
     const int64_t blk0 = g.tin * kDqBlock;
 #pragma unroll
@@ -375,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       if (lane == 0) p.partials[p.tile_base + tile] = make_double2(se, sw);
     }
     if (L.packed) {
-      const uint8_t* os = smem + kOutOff + buf * kPackedTileBytes;
+      const uint8_t* os = smem + kOutOff;
       uint8_t* gp = L.packed + g.tin * kPackedTileBytes;
       if (g.cnt == kTile) {
 #pragma unroll
@@ -390,6 +391,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         }
       }
     }
+    __syncthreads();  // the single output and reduction buffers are free again
   }
 
   if (aborted && t == 0) {
