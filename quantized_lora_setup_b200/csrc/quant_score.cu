@@ -40,6 +40,8 @@ namespace {
 constexpr int kBpt = 2;
 constexpr int kThreads = kDqBlock / kBpt;  // a CTA covers one tile (= one DQ block)
 constexpr int kWarps = kThreads / 32;
+// chunk loop of the coding pass unrolled by 2: smaller code, slightly faster than full unroll
+constexpr int kP2Unroll = 2;
 constexpr int kCtasPerSm = 4;  // 44 KB of shared memory and 128 registers per thread, no spills
 constexpr int kMaxLayersPerLaunch = 384;
 
@@ -261,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     for (int b = 0; b < kBpt; ++b) es2[b] = ws2[b] = make_float2(0.0f, 0.0f);
     const float2 scale2 = make_float2(15.5f, 15.5f), off2 = make_float2(8388624.0f, 8388624.0f);
     uint8_t* ost = smem + kOutOff;
-#pragma unroll
+#pragma unroll kP2Unroll
     for (int k2 = 0; k2 < 8; ++k2) {
       const int c = (k2 + rot) & 7;
 #pragma unroll
