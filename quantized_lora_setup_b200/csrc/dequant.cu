@@ -12,13 +12,14 @@
 // 8 x 32 chunks for memory-level parallelism.  The level lookup is a warp shuffle whose
 // source lane is the nibble itself (lanes 16..31 mirror 0..15, so the shifted word needs
 // no mask).  fl(c / 255) for the 256 possible bytes is tabulated in shared memory with a
-// correctly rounded divide.
+// correctly rounded divide.  Stores are streaming (evict-first), which the write-heavy
+// traffic favours.
 #include "device.cuh"
 
 namespace aqnf4 {
 namespace {
 
-constexpr int kChunksPerLane = 8;
+constexpr int kChunksPerLane = 8;  // 16 costs occupancy (108 registers), 4 too few loads in flight
 
 struct DqParams {
   float level[16];
@@ -80,7 +81,8 @@ __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ pac
       }
       const int64_t c = g * kGroup + j * 32 + lane;
       if (c < full_chunks) {
-        *reinterpret_cast<uint4*>(out + 8 * c) = make_uint4(o[0], o[1], o[2], o[3]);
+        // streaming store: the output is not read again by this kernel
+        __stcs(reinterpret_cast<uint4*>(out + 8 * c), make_uint4(o[0], o[1], o[2], o[3]));
       } else if (c < nchunk) {
         for (int e = 0; e < 8 && 8 * c + e < n; ++e)
           out[8 * c + e] = static_cast<uint16_t>(o[e >> 1] >> ((e & 1) * 16));
