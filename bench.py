@@ -43,6 +43,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dequant", action="store_true")
+    ap.add_argument("--extra-workloads", default="14b,1.4b",
+                    help="comma-separated workloads also timed (1 GPU only; '' to skip)")
     ap.add_argument("--max-layers", type=int, default=0,
                     help="use only the first N layers (small cases for profiling)")
     return ap.parse_args()
@@ -380,12 +382,76 @@ def run_native(args):
                       f"{len(sample)} layers ({elems} weights), quantize + DQ + error, one "
                       f"thread per slice"}
 
+    extras = [w for w in args.extra_workloads.split(",") if w and w != args.workload]
+    if world == 1 and extras:
+        del weights, stor, descs, ws
+        torch.cuda.empty_cache()
+        result["workloads"] = {name: bench_workload(name, dev, stream, peak, steps=50)
+                               for name in extras}
+
     if world > 1:
         dist.barrier(device_ids=[local])
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
     return 0
+
+
+def bench_workload(name, dev, stream, peak, steps):
+    """The same scoring step on another model shape (1 GPU): GB/s of weights read, the fused
+    kernel's roofline fraction, and the selection at every budget of that workload."""
+    import torch
+
+    from quantized_lora_setup_b200 import aqnf4, synth
+    wl = synth.workload(name)
+    weights = [synth.layer_device(s, wl.seed, i, dev) for i, s in enumerate(wl.layers)]
+    stor = [aqnf4.NF4Storage(w.numel(), dev) for w in weights]
+    descs = aqnf4.make_layers([{"w": w, "packed": s.packed, "codes8": s.codes8,
+                                "scales": s.scales} for w, s in zip(weights, stor)])
+    ws = torch.empty(max(256, aqnf4.aqnf4_workspace_size(descs)), dtype=torch.uint8, device=dev)
+    L = len(weights)
+    se = torch.empty(L, dtype=torch.float64, device=dev)
+    sw = torch.empty_like(se)
+    rel = torch.empty(L, dtype=torch.float32, device=dev)
+    cost = torch.tensor([aqnf4.aqnf4_cost_bytes(s.numel) for s in wl.layers], dtype=torch.int64,
+                        device=dev)
+    sel = torch.empty(L, dtype=torch.int32, device=dev)
+    kout = torch.empty(1, dtype=torch.int32, device=dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+
+    def step(e=None):
+        if e is not None:
+            e[0].record(stream)
+        aqnf4.aqnf4_layer_error(descs, ws, se, sw, rel, None, stream)
+        if e is not None:
+            e[1].record(stream)
+        aqnf4.aqnf4_select_topk(rel, cost, wl.budgets[0], wl.k_cap, sel, kout, stream)
+
+    for _ in range(3):
+        step()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    a.record(stream)
+    for e in evs:
+        step(e)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b) / steps
+    kern_ms = statistics.mean(x.elapsed_time(y) for x, y in evs)
+    alg = sum(algorithmic_bytes(w.numel()) for w in weights)
+    kept = {}
+    for budget in wl.budgets:
+        aqnf4.aqnf4_select_topk(rel, cost, budget, wl.k_cap, sel, kout, stream)
+        kept[str(budget)] = int(kout.item())
+    achieved = alg / (kern_ms / 1e3) / 1e9
+    dts = sorted({str(s.dtype).replace("torch.", "") for s in wl.layers})
+    return {"workload": workload_desc(wl), "dtype_in": "/".join(dts), "steps": steps,
+            "ms_per_step": ms, "value": wl.weight_bytes / (ms / 1e3) / 1e9, "unit": UNIT,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "kernel": "k_quant_score",
+                         "launch_ms": kern_ms, "alg_bytes_per_launch": alg},
+            "kept_per_budget": kept}
 
 
 def bench_dequant(dev, stream, peak):

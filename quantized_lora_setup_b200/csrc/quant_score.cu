@@ -353,8 +353,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     for (int b = 0; b < kBpt; ++b) {
       const int blk = t + b * kThreads;
       if (blk < nblk) {
-        if (L.absmax) L.absmax[blk0 + blk] = a[b];
-        if (L.codes8) L.codes8[blk0 + blk] = dq_code(a[b], sdq);
+        if (L.absmax) __stcs(L.absmax + blk0 + blk, a[b]);
+        if (L.codes8) __stcs(reinterpret_cast<char*>(L.codes8) + blk0 + blk,
+                             static_cast<char>(dq_code(a[b], sdq)));
       }
     }
     if (t == 0 && L.codes8) {
@@ -383,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       if (g.cnt == kTile) {
 #pragma unroll
         for (int i = t; i < kPackedTileBytes / 16; i += kThreads)
-          *reinterpret_cast<uint4*>(gp + 16 * i) = lds128(os + 16 * i);
+          __stcs(reinterpret_cast<uint4*>(gp + 16 * i), lds128(os + 16 * i));
       } else {
         const int nbytes = (g.cnt + 1) >> 1;
         for (int i = t; i < nbytes; i += kThreads) {
