@@ -180,6 +180,15 @@ AQNF4_API aqnf4_status aqnf4_select_topk(const float* rel_err, const int64_t* co
                                int64_t budget_bytes, int32_t k_cap, int32_t* sel_idx,
                                int32_t* k_out, cudaStream_t stream);
 
+/* Diagnostic for failure detection (no counterpart on the pages).  Runs the bounded wait
+   that every bulk-copy consumer in this library uses, on an mbarrier that nothing ever
+   completes, with a limit of timeout_ns (1 ns .. 2 s; the kernels themselves use 2 s).  The
+   wait gives up, the kernel stores AQNF4_ERR_TIMEOUT in *dev_flag (device int32, required)
+   and, if waited_ns (device int64) is non-NULL, the nanoseconds it waited; then it returns
+   normally, leaving the context usable.  Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+AQNF4_API aqnf4_status aqnf4_selftest_wait_timeout(int64_t timeout_ns, int32_t* dev_flag,
+                                                   int64_t* waited_ns, cudaStream_t stream);
+
 /* Incremental bytes of keeping an n-element layer in 16 bits instead of its NF4 storage
    (packed + codes8 + scales): 2n - (ceil(n/2) + ceil(n/64) + 4*ceil(ceil(n/64)/256)).
    Host only; -1 for n < 1.  (The 0.2 GiB extra memory of the abstract's quality setting is

@@ -89,6 +89,8 @@ def library() -> ctypes.CDLL:
     lib.aqnf4_layer_error_noalloc.restype = st
     lib.aqnf4_select_topk.argtypes = [P, P, i32, i64, i32, P, P, P]
     lib.aqnf4_select_topk.restype = st
+    lib.aqnf4_selftest_wait_timeout.argtypes = [i64, P, P, P]
+    lib.aqnf4_selftest_wait_timeout.restype = st
     lib.aqnf4_cost_bytes.argtypes = [i64]
     lib.aqnf4_cost_bytes.restype = i64
     lib.aqnf4_launch_count.argtypes = []
@@ -207,6 +209,12 @@ def aqnf4_select_topk(rel_err: torch.Tensor, cost_bytes: torch.Tensor, budget_by
     _check(library().aqnf4_select_topk(_ptr(rel_err), _ptr(cost_bytes), rel_err.numel(),
                                        int(budget_bytes), int(k_cap), _ptr(sel_idx), _ptr(k_out),
                                        _stream(stream)), "aqnf4_select_topk")
+
+
+def aqnf4_selftest_wait_timeout(timeout_ns: int, dev_flag: torch.Tensor,
+                                waited_ns: Optional[torch.Tensor] = None, stream=None) -> None:
+    _check(library().aqnf4_selftest_wait_timeout(int(timeout_ns), _ptr(dev_flag), _ptr(waited_ns),
+                                                 _stream(stream)), "aqnf4_selftest_wait_timeout")
 
 
 def aqnf4_cost_bytes(n: int) -> int:

@@ -15,7 +15,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIB_DIR, "libaqnf4.so")
-SOURCES = ["codebook.cpp", "quant_score.cu", "double_quant.cu", "dequant.cu", "select.cu"]
+SOURCES = ["codebook.cpp", "quant_score.cu", "double_quant.cu", "dequant.cu", "select.cu",
+           "selftest.cu"]
 HEADERS = ["internal.h", "device.cuh"]
 
 NVCC_FLAGS = [

@@ -131,6 +131,11 @@ def test_argument_checks_return_before_any_launch(lib):
     assert lib.aqnf4_select_topk(V(0x100), V(0x200), 5, -1, -1, V(0x300), V(0x400), None) == aqnf4.AQNF4_ERR_INVALID_ARG
     assert lib.aqnf4_select_topk(V(0x100), V(0x200), 0, 10, -1, V(0x300), V(0x400), None) == aqnf4.AQNF4_ERR_INVALID_ARG
     assert lib.aqnf4_select_topk(V(0x100), V(0x204), 5, 10, -1, V(0x300), V(0x400), None) == aqnf4.AQNF4_ERR_ALIGNMENT
+    # bounded-wait diagnostic
+    assert lib.aqnf4_selftest_wait_timeout(0, V(0x100), None, None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert lib.aqnf4_selftest_wait_timeout(3_000_000_000, V(0x100), None, None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert lib.aqnf4_selftest_wait_timeout(1000, None, None, None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert lib.aqnf4_selftest_wait_timeout(1000, V(0x102), None, None) == aqnf4.AQNF4_ERR_ALIGNMENT
     assert lib.aqnf4_launch_count() == before
 
 

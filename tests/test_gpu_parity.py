@@ -275,3 +275,18 @@ def test_select_topk_matches_oracle(cuda, seed):
     assert got[: k.item()].tolist() == ref
     full = oracle.select_topk(e, np.zeros(L, np.int64), 0, -1)
     assert got.tolist() == full  # the whole ranking is returned
+
+
+def test_bounded_wait_gives_up_and_reports(cuda):
+    """A wait on an mbarrier nothing completes ends with AQNF4_ERR_TIMEOUT, not a hang, and the
+    context keeps working afterwards."""
+    flag = torch.zeros(1, dtype=torch.int32, device=cuda)
+    waited = torch.zeros(1, dtype=torch.int64, device=cuda)
+    aqnf4.aqnf4_selftest_wait_timeout(20_000_000, flag, waited)  # 20 ms
+    torch.cuda.synchronize()
+    assert flag.item() == aqnf4.AQNF4_ERR_TIMEOUT
+    assert 20_000_000 <= waited.item() < 2_000_000_000
+    # the device is still usable: a normal call right after succeeds and is correct
+    w = synth.random_bits_host(1000, seed=5, dtype=torch.bfloat16)
+    packed, _ = aqnf4.quantize(w.to(cuda))
+    assert np.array_equal(packed.cpu().numpy(), oracle.quantize(bits(w), oracle.BF16)[0])
