@@ -195,6 +195,16 @@ AQNF4_API aqnf4_status aqnf4_selftest_wait_timeout(int64_t timeout_ns, int32_t* 
    read as a budget on this quantity.) */
 AQNF4_API int64_t aqnf4_cost_bytes(int64_t n);
 
+/* The fused pass's code lookup, for inspection (host only; no counterpart on the pages,
+   which define the code as the nearest level, i.e. the number of midpoints below v).
+   curve[2] = (a, b); slot_mid[32], slot_level[32].  For a normalised value v with
+   |v| <= 1 + 2^-20 the kernels compute, in binary32, s = fma(v*v, b, a) and
+   k = round_to_nearest(fma(v, s, 2^23 + 8)) - 2^23, and take
+   code = k - 1 + (v > slot_mid[k]) and level = slot_level[code + 1].  The library checks
+   when it builds the tables that this equals the midpoint count for every such v.
+   Host arrays, caller-owned.  Errors: INVALID_ARG (null pointer), CUDA (tables failed). */
+AQNF4_API aqnf4_status aqnf4_slot_tables(float* curve, float* slot_mid, float* slot_level);
+
 /* Number of kernels this library has launched in this process (host counter). */
 AQNF4_API uint64_t aqnf4_launch_count(void);
 

@@ -91,6 +91,8 @@ def library() -> ctypes.CDLL:
     lib.aqnf4_select_topk.restype = st
     lib.aqnf4_selftest_wait_timeout.argtypes = [i64, P, P, P]
     lib.aqnf4_selftest_wait_timeout.restype = st
+    lib.aqnf4_slot_tables.argtypes = [P, P, P]
+    lib.aqnf4_slot_tables.restype = st
     lib.aqnf4_cost_bytes.argtypes = [i64]
     lib.aqnf4_cost_bytes.restype = i64
     lib.aqnf4_launch_count.argtypes = []
@@ -215,6 +217,19 @@ def aqnf4_selftest_wait_timeout(timeout_ns: int, dev_flag: torch.Tensor,
                                 waited_ns: Optional[torch.Tensor] = None, stream=None) -> None:
     _check(library().aqnf4_selftest_wait_timeout(int(timeout_ns), _ptr(dev_flag), _ptr(waited_ns),
                                                  _stream(stream)), "aqnf4_selftest_wait_timeout")
+
+
+def aqnf4_slot_tables():
+    """(curve float32[2], slot_mid float32[32], slot_level float32[32]) of the fused pass."""
+    import numpy as np
+    curve = np.zeros(2, np.float32)
+    slot_mid = np.zeros(32, np.float32)
+    slot_level = np.zeros(32, np.float32)
+    _check(library().aqnf4_slot_tables(curve.ctypes.data_as(ctypes.c_void_p),
+                                       slot_mid.ctypes.data_as(ctypes.c_void_p),
+                                       slot_level.ctypes.data_as(ctypes.c_void_p)),
+           "aqnf4_slot_tables")
+    return curve, slot_mid, slot_level
 
 
 def aqnf4_cost_bytes(n: int) -> int:

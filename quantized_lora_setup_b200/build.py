@@ -1,8 +1,8 @@
 """Build libaqnf4.so (the C-ABI library) in-tree for sm_100a with nvcc.
 
 ``python -m quantized_lora_setup_b200.build`` or ``build()``; the shared library lands in
-``quantized_lora_setup_b200/lib/libaqnf4.so``.  No fast-math: the kernels rely on IEEE
-rounding for bit-exact NF4 codes.
+``quantized_lora_setup_b200/lib/libaqnf4.so``.  No fast-math and no implicit FMA
+contraction: the kernels rely on IEEE rounding, exactly as written, for bit-exact NF4 codes.
 """
 import os
 import shutil
@@ -19,9 +19,12 @@ SOURCES = ["codebook.cpp", "quant_score.cu", "double_quant.cu", "dequant.cu", "s
            "selftest.cu"]
 HEADERS = ["internal.h", "device.cuh"]
 
+# -fmad=false: no multiply and add is ever fused behind the code's back (every FMA the
+# kernels want is written out).  A fused x*r - mid decides ties against the exact product
+# instead of the rounded v = fl(x*r) and flips codes where v equals a midpoint exactly.
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
-    "-O3", "-lineinfo", "-std=c++17",
+    "-O3", "-lineinfo", "-std=c++17", "-fmad=false",
     "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
     "--shared", "-cudart", "static",
 ]

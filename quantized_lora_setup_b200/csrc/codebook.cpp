@@ -41,24 +41,47 @@ Tables g_tables;
 const Tables* g_tables_ptr = nullptr;
 std::once_flag g_tables_once;
 
+// Slot curve k(v) = round(a v + b v^3 + 8) for the default codebook: the max-margin odd
+// cubic (both coefficients exact in binary32).  check_slot_curve proves it below.
+constexpr float kCurveA = 11.71875f;
+constexpr float kCurveB = -4.125f;
+
+// h(v) = a v + b v^3 + 8.5; the kernel's round-to-nearest of a v + b v^3 + 8 is floor(h)
+// away from ties, and either neighbour at a tie.  For v in (mid_{j-1}, mid_j] (with the
+// ends -1 - 2^-20 and 1 + 2^-20 outside the first and last midpoints) the slot must be j or
+// j + 1, i.e. j + margin <= h(v) <= j + 2 - margin.  A cubic's extremes on an interval are
+// at its ends or its critical points, so checking those points in binary64 is a proof; the
+// margin (1/64 of a slot) dwarfs the error of evaluating h in binary32 (below 1e-5).
+bool check_slot_curve(const Tables& t) {
+  const double a = t.curve_a, b = t.curve_b, margin = 1.0 / 64.0;
+  auto h = [&](double v) { return a * v + b * v * v * v + 8.5; };
+  const double ends = 1.0 + std::ldexp(1.0, -20);
+  const double crit = (b < 0.0 && a > 0.0) ? std::sqrt(a / (-3.0 * b)) : -1.0;
+  for (int j = 0; j < 16; ++j) {
+    const double lo = j == 0 ? -ends : t.mid[j - 1];
+    const double hi = j == 15 ? ends : t.mid[j];
+    double hmin = std::fmin(h(lo), h(hi)), hmax = std::fmax(h(lo), h(hi));
+    for (double c : {crit, -crit}) {
+      if (crit > 0.0 && c > lo && c < hi) {
+        hmin = std::fmin(hmin, h(c));
+        hmax = std::fmax(hmax, h(c));
+      }
+    }
+    if (hmin < j + margin || hmax > j + 2 - margin) return false;
+  }
+  return true;
+}
+
 bool build_tables(Tables& t) {
   if (aqnf4_codebook(0.0, t.level, t.mid) != AQNF4_OK) return false;
-  int bucket_of_mid[15];
-  for (int j = 0; j < 15; ++j) {
-    // 15.5 * m has at most 29 significant bits for a binary32 m, so this is exact.
-    double pos = 15.5 * static_cast<double>(t.mid[j]) + 16.0;
-    bucket_of_mid[j] = static_cast<int>(std::floor(pos));
-    if (bucket_of_mid[j] < 0 || bucket_of_mid[j] > 31) return false;
-    if (j > 0 && bucket_of_mid[j] <= bucket_of_mid[j - 1]) return false;  // <= 1 per bucket
-  }
-  for (int b = 0; b < 32; ++b) {
-    t.bucket_mid[b] = std::numeric_limits<float>::infinity();
-    uint32_t below = 0;
-    for (int j = 0; j < 15; ++j) {
-      if (bucket_of_mid[j] < b) ++below;
-      if (bucket_of_mid[j] == b) t.bucket_mid[b] = t.mid[j];
-    }
-    t.bucket_code[b] = below;
+  t.curve_a = kCurveA;
+  t.curve_b = kCurveB;
+  if (!check_slot_curve(t)) return false;
+  for (int k = 0; k < 32; ++k) {
+    t.slot_mid[k] = k == 0    ? -std::numeric_limits<float>::infinity()
+                    : k <= 15 ? t.mid[k - 1]
+                              : std::numeric_limits<float>::infinity();
+    t.slot_level[k] = k == 0 ? t.level[0] : k <= 16 ? t.level[k - 1] : t.level[15];
   }
   return true;
 }
@@ -126,6 +149,19 @@ int64_t aqnf4_cost_bytes(int64_t n) {
   const int64_t nb = (n + aqnf4::kBlock - 1) / aqnf4::kBlock;
   const int64_t nd = (nb + aqnf4::kDqBlock - 1) / aqnf4::kDqBlock;
   return 2 * n - ((n + 1) / 2 + nb + 4 * nd);
+}
+
+aqnf4_status aqnf4_slot_tables(float* curve, float* slot_mid, float* slot_level) {
+  if (!curve || !slot_mid || !slot_level) return AQNF4_ERR_INVALID_ARG;
+  const aqnf4::Tables* tb = aqnf4::default_tables();
+  if (!tb) return AQNF4_ERR_CUDA;
+  curve[0] = tb->curve_a;
+  curve[1] = tb->curve_b;
+  for (int k = 0; k < 32; ++k) {
+    slot_mid[k] = tb->slot_mid[k];
+    slot_level[k] = tb->slot_level[k];
+  }
+  return AQNF4_OK;
 }
 
 uint64_t aqnf4_launch_count(void) { return aqnf4::g_launches.load(std::memory_order_relaxed); }

@@ -69,15 +69,15 @@ __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ pac
 #pragma unroll
     for (int j = 0; j < kChunksPerLane; ++j) {
       const uint32_t w = wd[j];
-      const float2 a2 = make_float2(ap[j], ap[j]);
+      const f32x2 a2 = pair(ap[j], ap[j]);
       uint32_t o[4];
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
         // byte h holds element 2h in its high nibble and element 2h+1 in its low nibble
         const float q0 = __shfl_sync(kFull, tab_level, static_cast<int>(w >> (8 * h + 4)));
         const float q1 = __shfl_sync(kFull, tab_level, static_cast<int>(w >> (8 * h)));
-        const float2 v = mul2_rn(make_float2(q0, q1), a2);
-        o[h] = F::pack_rn(v.x, v.y);
+        const f32x2 v = pmul_rn(pair(q0, q1), a2);
+        o[h] = F::pack_rn(pair_lo(v), pair_hi(v));
       }
       const int64_t c = g * kGroup + j * 32 + lane;
       if (c < full_chunks) {

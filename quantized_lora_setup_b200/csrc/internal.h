@@ -17,17 +17,22 @@ constexpr int kTileBytes = kTile * 2;      // 16-bit weights of one tile
 constexpr int kPackedTileBytes = kTile / 2;
 
 // Lookup tables the kernels use, derived from the default codebook (codebook.cpp).
-//   level[c]    : NF4 level of code c (16 entries).
-//   bucket_mid  : for the bucket b = floor(15.5 v + 16) in [0, 32): the one midpoint that
-//                 falls in bucket b, or +inf when none does.
-//   bucket_code : number of midpoints below bucket b.
-// With these, #{ j : v > mid_j } = bucket_code[b] + (v > bucket_mid[b]) for every finite v
-// with |v| < 1 + 1/31 (every normalised value lies well inside that).
+//   level[c], mid[j] : the codebook (16 levels, 15 midpoints).
+//   curve_a, curve_b : the slot of a normalised value v is k(v) = round(a v + b v^3 + 8),
+//                      an odd cubic fitted so that every midpoint sits in a slot of its own:
+//                      for mid_{j-1} < v <= mid_j, k(v) is j or j + 1 (checked when the
+//                      tables are built, with a margin far above binary32 rounding).
+//   slot_mid[k]      : mid_{k-1} for k = 1..15; -inf at k = 0; +inf at k >= 16.
+//   slot_level[k]    : level[k-1] for k = 1..16 (lane k of a shuffle table); the unused
+//                      lanes repeat the end levels.
+// With these, #{ j : v > mid_j } = k(v) - 1 + (v > slot_mid[k(v)]) for every |v| <= 1 + 2^-20,
+// which covers every normalised value.  The code then indexes slot_level at k + 1.
 struct Tables {
   float level[16];
   float mid[15];
-  float bucket_mid[32];
-  uint32_t bucket_code[32];
+  float curve_a, curve_b;
+  float slot_mid[32];
+  float slot_level[32];
 };
 
 // Builds (once) and returns the tables of the default codebook.  Returns nullptr if the

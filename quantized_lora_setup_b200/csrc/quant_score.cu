@@ -20,9 +20,12 @@
 // tile into shared memory; four CTAs share an SM, so one CTA's copy overlaps the others'
 // arithmetic.  Each thread reads its blocks twice with conflict-free 16-byte loads (chunk
 // order rotated per thread): once for the absmax (packed bf16x2/f16x2 max), once to code,
-// the two blocks' work interleaved.  A code costs one round-toward-minus-infinity FMA
-// (bucket index), two warp-shuffle table lookups and one compare mask; two codes form a
-// packed byte directly, and the byte indexes the level shuffles.  Arithmetic on pairs uses
+// the two blocks' work interleaved.  A code does not count midpoints: an odd cubic
+// k = round(a v + b v^3 + 8) (three packed FMA-pipe instructions per two elements) puts
+// every midpoint in a slot of its own, so one warp-shuffle lookup of that slot's midpoint
+// and the sign of one subtract give code = k - 1 + (v > slot_mid[k]); the code then
+// indexes the level shuffle.  The tables and the proof that this equals the midpoint count
+// for every normalised v are built on the host (codebook.cpp).  Arithmetic on pairs uses
 // Blackwell's packed f32x2 instructions, and w_hat - x comes from the packed 16-bit w_hat
 // with one mixed-precision subtract.  Packed codes are staged in shared memory and leave with
 // coalesced 16-byte stores.  The per-tile extra work (the next bulk copy, the binary64
@@ -44,6 +47,13 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kP2Unroll = 2;
 constexpr int kCtasPerSm = 4;  // 44 KB of shared memory and 128 registers per thread, no spills
 constexpr int kMaxLayersPerLaunch = 384;
+
+// The coding loop keeps each code as c = bits(2^23 + slot) + (v > mid) = kCodeBias + code,
+// so that c's low 5 bits index the level table directly.  The byte (c0 << 4) + c1 and the
+// packed word sum_j byte_j << 8j then carry data-independent constants, removed once per word.
+constexpr uint32_t kCodeBias = 0x4B000001u;
+constexpr uint32_t kByteBias = (kCodeBias << 4) + kCodeBias;
+constexpr uint32_t kPackBias = kByteBias + (kByteBias << 8) + (kByteBias << 16) + (kByteBias << 24);
 
 // shared memory layout (bytes): one input stage, the packed-output stage, the per-block
 // (err, w^2, scale) floats, the per-warp absmax, the mbarrier and abort word.  The output
@@ -72,8 +82,9 @@ struct QParams {
   int64_t tile_base;   // index of this launch's first tile in the partials array
   double2* partials;   // per tile (sum (x - w_hat)^2, sum x^2); score only
   int32_t* flag;       // optional device status word
-  float bucket_mid[32];
-  uint32_t bucket_code[32];
+  float curve_a, curve_b;
+  float slot_mid[32];
+  float slot_level[32];
   float level[16];
   float mid[15];
   int32_t tile_begin[kMaxLayersPerLaunch + 1];  // first tile of each layer (launch-local)
@@ -134,8 +145,8 @@ __device__ __forceinline__ void issue_tile(const QParams& p, int64_t tile, uint8
   }
 }
 
-// Generic per-element path for a block whose absmax is 0, below the binary32 normal range,
-// or not finite.  Re-reads the block (natural element order) from shared memory, rewrites
+// Generic per-element path for a block whose absmax lies outside [2^-40, 2^40] (zero,
+// subnormal, huge or not finite).  Re-reads the block (natural element order) from shared memory, rewrites
 // this thread's packed words and returns the normalised sums (err, w^2) -- scaled by a^2
 // later like the fast path's.
 template <int DT, bool SCORE>
@@ -195,10 +206,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   // this lane's entries of the shuffle lookup tables
-  const float tab_mid = p.bucket_mid[lane];
-  const uint32_t tab_code = p.bucket_code[lane];
-  const uint32_t tab_code16 = tab_code << 4;  // the same, already in the high nibble
-  const float tab_level = p.level[lane & 15];  // lanes 16..31 mirror 0..15
+  const float tab_mid = p.slot_mid[lane];
+  const float tab_level = p.slot_level[lane];
 
   if (t == 0) {
     mbar_init(bar_a, 1);
@@ -236,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
     // ---- pass 1: absmax of this thread's blocks (NaN propagates)
     float a[kBpt], r[kBpt];
-    bool fast[kBpt], fast_sum[kBpt];
+    bool fast[kBpt];
 #pragma unroll
     for (int b = 0; b < kBpt; ++b) {
       const uint8_t* my = stage + (t + b * kThreads) * 128;
@@ -250,18 +259,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       m0 = F::absmax2(m0, m1);
       m0 = F::absmax2(m0, __byte_perm(m0, 0, 0x1032));
       a[b] = F::abs_lo(m0);
-      fast[b] = (a[b] >= 0x1p-126f) && (a[b] <= FLT_MAX);
       // 2^-40 <= a <= 2^40: (w_hat - x)^2 and x^2 cannot overflow or flush in binary32
-      fast_sum[b] = (a[b] >= 0x1p-40f) && (a[b] <= 0x1p40f);
+      fast[b] = (a[b] >= 0x1p-40f) && (a[b] <= 0x1p40f);
       r[b] = fast[b] ? __frcp_rn(a[b]) : 0.0f;
     }
 
     // ---- pass 2: codes, packing, error; the blocks' chains interleave (all lanes run this
     // so the shuffles stay converged)
-    float2 es2[kBpt], ws2[kBpt];
+    f32x2 es2[kBpt], ws2[kBpt], r2[kBpt], a2[kBpt];
 #pragma unroll
-    for (int b = 0; b < kBpt; ++b) es2[b] = ws2[b] = make_float2(0.0f, 0.0f);
-    const float2 scale2 = make_float2(15.5f, 15.5f), off2 = make_float2(8388624.0f, 8388624.0f);
+    for (int b = 0; b < kBpt; ++b) {
+      es2[b] = ws2[b] = pair(0.0f, 0.0f);
+      r2[b] = pair(r[b], r[b]);
+      a2[b] = pair(a[b], a[b]);
+    }
+    const f32x2 ca2 = pair(p.curve_a, p.curve_a), cb2 = pair(p.curve_b, p.curve_b);
+    const f32x2 off2 = pair(8388616.0f, 8388616.0f);  // 2^23 + 8
     uint8_t* ost = smem + kOutOff;
 #pragma unroll kP2Unroll
     for (int k2 = 0; k2 < 8; ++k2) {
@@ -271,38 +284,41 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const int blk = t + b * kThreads;
         const uint4 v4 = lds128(stage + blk * 128 + c * 16);
         const uint32_t w4[4] = {v4.x, v4.y, v4.z, v4.w};
-        const float2 r2 = make_float2(r[b], r[b]), a2 = make_float2(a[b], a[b]);
         uint32_t pk = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const uint32_t wd = w4[j];
-          const float2 x = make_float2(F::lo(wd), F::hi(wd));
-          const float2 v = mul2_rn(x, r2);
-          // floor(15.5 v + 16) lands in the low 5 bits of tt (2^23 <= tt < 2^23 + 32)
-          const float2 tt = fma2_rm(v, scale2, off2);
-          const int i0 = __float_as_int(tt.x), i1 = __float_as_int(tt.y);
-          const float m0s = __shfl_sync(kFull, tab_mid, i0);
-          const float m1s = __shfl_sync(kFull, tab_mid, i1);
-          // byte = code0 << 4 | code1 = (base0 << 4) + base1 + [v0 > m0] * 16 + [v1 > m1]
-          const uint32_t base =
-              __shfl_sync(kFull, tab_code16, i0) + __shfl_sync(kFull, tab_code, i1);
-          const uint32_t byte = base - 16u * static_cast<uint32_t>(gt_mask(v.x, m0s)) -
-                                static_cast<uint32_t>(gt_mask(v.y, m1s));
+          const f32x2 x = pair(F::lo(wd), F::hi(wd));
+          const f32x2 v = pmul_rn(x, r2[b]);
+          // slot k = round(a v + b v^3 + 8) lands in the low 5 bits of kk = 2^23 + k
+          const f32x2 kk = pfma_rn(v, pfma_rn(pmul_rn(v, v), cb2, ca2), off2);
+          const uint32_t k0 = __float_as_uint(pair_lo(kk)), k1 = __float_as_uint(pair_hi(kk));
+          const f32x2 mid =
+              pair(__shfl_sync(kFull, tab_mid, static_cast<int>(k0)),
+                   __shfl_sync(kFull, tab_mid, static_cast<int>(k1)));
+          // v > mid exactly when fl(mid - v) is negative (a difference is exact in sign).
+          // This needs the rounded v: were the multiply fused into the subtract (x r - mid,
+          // which ptxas does for a product with no other use, despite .rn), ties v == mid
+          // would follow the exact product.  Here v also feeds the slot curve, and the GPU
+          // parity tests include blocks of exact ties.
+          const f32x2 dm = psub_rn(mid, v);
+          // c = bits(kk) + (v > mid) = kCodeBias + code: code + 1 in the low 5 bits
+          const uint32_t c0 = k0 + (__float_as_uint(pair_lo(dm)) >> 31);
+          const uint32_t c1 = k1 + (__float_as_uint(pair_hi(dm)) >> 31);
+          const uint32_t byte = (c0 << 4) + c1;  // code0 << 4 | code1, plus kByteBias
           pk = j == 0 ? byte : pk + (byte << (8 * j));
           if (SCORE) {
-            // the level tables mirror lanes 16..31, so the low 5 bits of byte (code1 and one
-            // bit of code0) and of byte >> 4 (code0) pick the right levels
-            const float q0 = __shfl_sync(kFull, tab_level, static_cast<int>(byte >> 4));
-            const float q1 = __shfl_sync(kFull, tab_level, static_cast<int>(byte));
-            const float2 wq = mul2_rn(make_float2(q0, q1), a2);
-            const uint32_t hb = F::pack_rn(wq.x, wq.y);
+            const float q0 = __shfl_sync(kFull, tab_level, static_cast<int>(c0));
+            const float q1 = __shfl_sync(kFull, tab_level, static_cast<int>(c1));
+            const f32x2 wq = pmul_rn(pair(q0, q1), a2[b]);
+            const uint32_t hb = F::pack_rn(pair_lo(wq), pair_hi(wq));
             // w_hat - x straight from the packed 16-bit w_hat (the sign does not matter)
-            const float2 d = make_float2(F::sub_lo(hb, x.x), F::sub_hi(hb, x.y));
-            es2[b] = fma2_rn(d, d, es2[b]);
-            ws2[b] = fma2_rn(x, x, ws2[b]);
+            const f32x2 d = pair(F::sub_lo(hb, pair_lo(x)), F::sub_hi(hb, pair_hi(x)));
+            es2[b] = pfma_rn(d, d, es2[b]);
+            ws2[b] = pfma_rn(x, x, ws2[b]);
           }
         }
-        *reinterpret_cast<uint32_t*>(ost + blk * 32 + c * 4) = pk;
+        *reinterpret_cast<uint32_t*>(ost + blk * 32 + c * 4) = pk - kPackBias;
       }
     }
 
@@ -314,10 +330,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
     for (int b = 0; b < kBpt; ++b) {
       const int blk = t + b * kThreads;
-      float2 sums = make_float2(es2[b].x + es2[b].y, ws2[b].x + ws2[b].y);
+      float2 sums = make_float2(pair_lo(es2[b]) + pair_hi(es2[b]),
+                                pair_lo(ws2[b]) + pair_hi(ws2[b]));
       // factor that turns this block's sums into weight units once squared
       float sum_scale = 1.0f;
-      if (!fast[b] || !fast_sum[b]) {
+      if (!fast[b]) {
         sums = block_generic<DT, SCORE>(stage + blk * 128, a[b], p, ost + blk * 32);
         sum_scale = a[b];
       }
@@ -467,9 +484,11 @@ cudaError_t launch_main_dt(int dt, bool score, const QParams& p, cudaStream_t st
 }
 
 void fill_tables(QParams& p, const Tables& tb) {
+  p.curve_a = tb.curve_a;
+  p.curve_b = tb.curve_b;
   for (int i = 0; i < 32; ++i) {
-    p.bucket_mid[i] = tb.bucket_mid[i];
-    p.bucket_code[i] = tb.bucket_code[i];
+    p.slot_mid[i] = tb.slot_mid[i];
+    p.slot_level[i] = tb.slot_level[i];
   }
   for (int i = 0; i < 16; ++i) p.level[i] = tb.level[i];
   for (int i = 0; i < 15; ++i) p.mid[i] = tb.mid[i];

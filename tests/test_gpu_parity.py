@@ -290,3 +290,60 @@ def test_bounded_wait_gives_up_and_reports(cuda):
     w = synth.random_bits_host(1000, seed=5, dtype=torch.bfloat16)
     packed, _ = aqnf4.quantize(w.to(cuda))
     assert np.array_equal(packed.cpu().numpy(), oracle.quantize(bits(w), oracle.BF16)[0])
+
+
+def _midpoint_tie_blocks(dt):
+    """Blocks whose elements normalise exactly onto a codebook midpoint or one ulp beside it.
+
+    For every 16-bit block maximum a and every target m (each midpoint and its binary32
+    neighbours), the 16-bit values next to m * a are tried; those with fl(x * fl(1/a)) == m
+    are kept.  A block is [a, its ties..., zeros], so its absmax is a.  These are the inputs
+    where the code is decided by a comparison with no slack at all ("QLoRA", "How It Works":
+    the nearest level, with ties going to the lower one).  binary16 has about 150 such
+    elements; bfloat16 has none (with 8-bit significands x * fl(1/a) never lands on these
+    binary32 midpoints; the closest are about 11 ulps away), so only binary16 is tested.
+    """
+    levels, mids = oracle.codebook()
+    targets = np.concatenate([mids, np.nextafter(mids, np.float32(2)),
+                              np.nextafter(mids, np.float32(-2))]).astype(np.float32)
+    h = np.arange(0x8000, dtype=np.int64)
+    av = torch.from_numpy(h.astype(np.int16)).view(dt).float().numpy()
+    keep = np.isfinite(av) & (av >= 2.0 ** -126)
+    h, av = h[keep], av[keep]
+    r = (np.float32(1) / av).astype(np.float32)
+    est = (targets[None, :] * av[:, None]).astype(np.float32)          # (A, T)
+    est16 = torch.from_numpy(est).to(dt).view(torch.int16).numpy().astype(np.int64)
+    blocks = []
+    for d in (-1, 0, 1):
+        cand = est16 + np.where(est16 >= 0, d, -d)                      # magnitude neighbours
+        cand16 = (cand & 0xFFFF).astype(np.uint16).view(np.int16)
+        xv = torch.from_numpy(cand16).view(dt).float().numpy()
+        v = (xv * r[:, None]).astype(np.float32)
+        hit = (v == targets[None, :]) & (np.abs(xv) <= av[:, None])
+        for ai in np.nonzero(hit.any(1))[0]:
+            xs = xv[ai][hit[ai]]
+            blocks.append((av[ai], xs))
+    w = []
+    for a, xs in blocks:
+        for s in range(0, len(xs), 63):
+            body = np.zeros(63, np.float32)
+            part = xs[s:s + 63]
+            body[:len(part)] = part
+            w.append(np.concatenate([[a], body]))
+    return torch.from_numpy(np.concatenate(w).astype(np.float32)).to(dt)
+
+
+def test_quantize_exact_midpoint_ties(cuda):
+    dt = torch.float16
+    w = _midpoint_tie_blocks(dt)
+    assert w.numel() >= 64 * 200
+    packed, absmax = aqnf4.quantize(w.to(cuda))
+    op, oa, _ = oracle.quantize(bits(w), DT[dt])
+    assert np.array_equal(packed.cpu().numpy(), op)
+    assert same_float_bits(absmax.cpu().numpy(), oa)
+    stor = aqnf4.NF4Storage(w.numel(), cuda)
+    se, sw, rel = aqnf4.score_layers([w.to(cuda)], [stor])
+    assert np.array_equal(stor.packed.cpu().numpy(), op)
+    ose, osw, orel = oracle.layer_error(bits(w), DT[dt])
+    assert se.item() == pytest.approx(ose, rel=RTOL)
+    assert rel.item() == pytest.approx(orel, rel=RTOL)
