@@ -35,6 +35,8 @@ def load():
     lib.oracle_quantize.restype = None
     lib.oracle_layer_error.argtypes = [P, ctypes.c_int, i64, P, P, P, P, P]
     lib.oracle_layer_error.restype = None
+    lib.oracle_layer_error_dq.argtypes = [P, ctypes.c_int, i64, P, P, P, P, P]
+    lib.oracle_layer_error_dq.restype = ctypes.c_int
     lib.oracle_double_quant.argtypes = [P, i64, P, P, P]
     lib.oracle_double_quant.restype = None
     lib.oracle_dequantize.argtypes = [P, P, P, P, i64, ctypes.c_int, P, P]
@@ -105,6 +107,19 @@ def layer_error(w, dtype, book=None):
     return float(se[0]), float(sw[0]), float(rel[0])
 
 
+def layer_error_dq(w, dtype, book=None):
+    """(sq_err, sq_w, rel_err) of one layer reconstructed from double-quantized constants."""
+    w = _as_bits(w).reshape(-1)
+    levels, mids = book if book is not None else codebook()
+    se = np.zeros(1, np.float64)
+    sw = np.zeros(1, np.float64)
+    rel = np.zeros(1, np.float32)
+    if load().oracle_layer_error_dq(_ptr(w), dtype, w.size, _ptr(levels), _ptr(mids), _ptr(se),
+                                    _ptr(sw), _ptr(rel)) != 0:
+        raise MemoryError("oracle_layer_error_dq")
+    return float(se[0]), float(sw[0]), float(rel[0])
+
+
 def double_quant(absmax):
     """8-bit / 256-block double quantization: (codes8 uint8[nb], scales float32[ceil(nb/256)], nonfinite)."""
     absmax = np.ascontiguousarray(absmax, np.float32).reshape(-1)
@@ -161,6 +176,7 @@ def dtype_bits_to_f32(bits, dtype):
 
 
 __all__ = ["F16", "BF16", "load", "default_pmax", "codebook", "quantize", "layer_error",
+           "layer_error_dq",
            "double_quant", "dequantize", "cost_bytes", "select_topk", "f32_to_dtype_bits",
            "dtype_bits_to_f32"]
 

@@ -44,12 +44,16 @@
  *   - reconstruction: w_hat = dtype_rn(fl(q[code] * a)); the layer score is
  *     sqrt(sum (x - w_hat)^2 / sum x^2), sums in binary64 in element order.
  *   - double quantization: per 256 constants s = max a; code8 = rint_even(fl(fl(a/s)*255)).
+ *   - the DQ-absmax score (an option): the same error with w_hat reconstructed from the
+ *     double-quantized constant a' = fl(fl(code8/255) * s) -- what a stored NF4 + DQ model
+ *     dequantizes to -- while the codes still come from the binary32 absmax.
  *   - selection: sort by (score desc, index asc, NaN last); keep the longest prefix with
  *     at most k_cap layers and total incremental cost <= budget.
  */
 #include <fenv.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #define OR_F16 0
@@ -320,6 +324,61 @@ void oracle_double_quant(const float* absmax, int64_t nb, uint8_t* codes8, float
       codes8[start + i] = (uint8_t)c;
     }
   }
+}
+
+/* ------------------------------------------------ DQ-absmax layer error */
+
+/* The layer error of a stored NF4 + DQ model ([QLoRA/HIW]: the constants are quantized in
+   turn and the weights are dequantized from them).  In order: (1) the binary32 absmax of
+   every block; (2) double quantization of those constants (oracle_double_quant); (3) each
+   block's reconstruction constant a' = fl(fl(code8/255) * s); (4) codes from the binary32
+   absmax, as in oracle_quantize; (5) w_hat = dtype_rn(fl(q[code] * a')) and the sums of
+   oracle_layer_error.  Returns 0, or -1 if memory runs out. */
+int oracle_layer_error_dq(const uint16_t* w, int dtype, int64_t n, const float levels[16],
+                          const float mids[15], double* sq_err, double* sq_w, float* rel) {
+  int64_t nb = (n + OR_BLOCK - 1) / OR_BLOCK;
+  int64_t nd = (nb + OR_DQ_BLOCK - 1) / OR_DQ_BLOCK;
+  float* absmax = (float*)calloc((size_t)nb, sizeof(float));
+  uint8_t* codes8 = (uint8_t*)calloc((size_t)nb, 1);
+  float* scales = (float*)calloc((size_t)nd, sizeof(float));
+  if (!absmax || !codes8 || !scales) {
+    free(absmax);
+    free(codes8);
+    free(scales);
+    return -1;
+  }
+  for (int64_t b = 0; b < nb; ++b) {
+    int64_t start = b * OR_BLOCK;
+    int len = (int)(n - start < OR_BLOCK ? n - start : OR_BLOCK);
+    absmax[b] = or_block_absmax(w, dtype, start, len);
+  }
+  oracle_double_quant(absmax, nb, codes8, scales, NULL);
+  int codes[OR_BLOCK];
+  double se = 0.0, sw = 0.0;
+  for (int64_t b = 0; b < nb; ++b) {
+    int64_t start = b * OR_BLOCK;
+    int len = (int)(n - start < OR_BLOCK ? n - start : OR_BLOCK);
+    float frac = (float)codes8[b] / 255.0f;
+    float a_dq = frac * scales[b / OR_DQ_BLOCK];
+    or_block_codes(w, dtype, start, len, absmax[b], mids, codes);
+    for (int i = 0; i < len; ++i) {
+      float x = or_load(w[start + i], dtype);
+      float prod = levels[codes[i]] * a_dq;
+      float what = or_load(or_round_to_dtype(prod, dtype), dtype);
+      double d = (double)x - (double)what;
+      se += d * d;
+      sw += (double)x * (double)x;
+    }
+  }
+  free(absmax);
+  free(codes8);
+  free(scales);
+  *sq_err = se;
+  *sq_w = sw;
+  double e = sw == 0.0 ? 0.0 : sqrt(se / sw);
+  if (isnan(se) || isnan(sw)) e = NAN;
+  *rel = (float)e;
+  return 0;
 }
 
 /* ------------------------------------------------------------- dequantize */

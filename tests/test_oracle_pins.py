@@ -374,6 +374,58 @@ def test_dequant_reconstructs_layer_error(book):
     assert se == pytest.approx(float(np.sum((x - deq) ** 2)), rel=1e-12)
 
 
+@pytest.mark.parametrize("dtype", [oracle.F16, oracle.BF16])
+def test_dq_layer_error_is_the_error_of_the_dequantized_model(book, dtype):
+    """The DQ-absmax score equals the error of what aqnf4_dequantize rebuilds from
+    packed codes + codes8 + scales (3 DQ blocks, ragged tail), summed here in numpy."""
+    rng = np.random.default_rng(21)
+    n = 64 * 700 + 13
+    tdt = torch.float16 if dtype == oracle.F16 else torch.bfloat16
+    z = rng.standard_normal(n) * np.repeat(rng.uniform(0.005, 0.05, n // 64 + 1), 64)[:n]
+    w = torch.from_numpy(z.astype(np.float32)).to(tdt)
+    bits = bits_of(w)
+    packed, absmax, _ = oracle.quantize(bits, dtype)
+    codes8, scales, _ = oracle.double_quant(absmax)
+    deq = oracle.dequantize(packed, n, dtype, codes8=codes8, scales=scales)
+    deq = torch.from_numpy(deq.view(np.int16)).view(tdt).double().numpy()
+    x = w.double().numpy()
+    se, sw, rel = oracle.layer_error_dq(bits, dtype)
+    assert se == pytest.approx(float(np.sum((x - deq) ** 2)), rel=1e-12)
+    assert sw == oracle.layer_error(bits, dtype)[1]
+    assert rel == pytest.approx(math.sqrt(se / sw), rel=1e-6)
+    # and it is not the plain score: the DQ constants differ from the binary32 absmax
+    assert se != oracle.layer_error(bits, dtype)[0]
+
+
+def test_dq_layer_error_equals_plain_when_constants_survive(book):
+    """Every block holding the same maximum A: code8 = 255 and a' = A, so both scores agree."""
+    rng = np.random.default_rng(22)
+    z = rng.uniform(-0.9, 0.9, (600, 64)).astype(np.float32) * 0.05
+    z[:, 5] = 0.05
+    w = torch.from_numpy(z.reshape(-1)).to(torch.bfloat16)
+    bits = bits_of(w)
+    assert oracle.layer_error_dq(bits, oracle.BF16) == oracle.layer_error(bits, oracle.BF16)
+
+
+def test_dq_layer_error_of_a_block_coded_to_zero(book):
+    """A block whose constant is below s/510 double-quantizes to 0, so a' = 0, w_hat = 0
+    and the block adds exactly its sum of squares to the error."""
+    rng = np.random.default_rng(23)
+    big = rng.uniform(-1.0, 1.0, 64).astype(np.float32)
+    big[0] = 1.0
+    small = (rng.uniform(-1.0, 1.0, 64) * 1e-3).astype(np.float32)
+    wb = torch.from_numpy(big).to(torch.bfloat16)
+    ws = torch.from_numpy(small).to(torch.bfloat16)
+    bits = np.concatenate([bits_of(wb), bits_of(ws)])
+    _, absmax, _ = oracle.quantize(bits, oracle.BF16)
+    codes8, _, _ = oracle.double_quant(absmax)
+    assert codes8.tolist() == [255, 0]
+    se, sw, _ = oracle.layer_error_dq(bits, oracle.BF16)
+    se_big = oracle.layer_error(bits_of(wb), oracle.BF16)[0]
+    xs = ws.double().numpy()
+    assert se == se_big + float(np.sum(xs * xs))
+
+
 # ---------------------------------------------------------------- selection
 
 
