@@ -43,6 +43,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dequant", action="store_true")
+    ap.add_argument("--no-dq-score", action="store_true",
+                    help="skip the step scored against the double-quantized constants")
     ap.add_argument("--extra-workloads", default="14b,1.4b",
                     help="comma-separated workloads also timed (1 GPU only; '' to skip)")
     ap.add_argument("--max-layers", type=int, default=0,
@@ -365,6 +367,10 @@ def run_native(args):
     if not args.no_dequant:
         result["dequant"] = bench_dequant(dev, stream, peak)
 
+    if world == 1 and not args.no_dq_score:
+        result["dq_score"] = bench_dq_score(weights, stor, wl, cost, budget, sel, k_sel, dev,
+                                            stream, peak, steps=min(K, 100))
+
     if not args.no_e2e:
         result["e2e"] = bench_e2e(args, weights, step, sel, kout, dev, stream, world,
                                   total_weight_bytes, L)
@@ -395,6 +401,57 @@ def run_native(args):
     if rank == 0:
         print(json.dumps(result), flush=True)
     return 0
+
+
+def bench_dq_score(weights, stor, wl, cost, budget, sel_plain, k_plain, dev, stream, peak, steps):
+    """The same scoring step with every layer scored against its double-quantized constants
+    (AQNF4_SCORE_DQ_ABSMAX): GB/s of weights read, the fused kernel's roofline fraction, and
+    whether the kept set under the budget differs from the plain score's."""
+    import torch
+
+    from quantized_lora_setup_b200 import aqnf4
+    descs = aqnf4.make_layers([{"w": w, "packed": s.packed, "codes8": s.codes8,
+                                "scales": s.scales, "flags": aqnf4.AQNF4_SCORE_DQ_ABSMAX}
+                               for w, s in zip(weights, stor)])
+    L = len(weights)
+    ws = torch.empty(max(256, aqnf4.aqnf4_workspace_size(descs)), dtype=torch.uint8, device=dev)
+    se = torch.empty(L, dtype=torch.float64, device=dev)
+    sw = torch.empty_like(se)
+    rel = torch.empty(L, dtype=torch.float32, device=dev)
+    sel = torch.empty(L, dtype=torch.int32, device=dev)
+    kout = torch.empty(1, dtype=torch.int32, device=dev)
+
+    def step(ev_a=None, ev_b=None):
+        if ev_a is not None:
+            ev_a.record(stream)
+        aqnf4.aqnf4_layer_error(descs, ws, se, sw, rel, None, stream)
+        if ev_b is not None:
+            ev_b.record(stream)
+        aqnf4.aqnf4_select_topk(rel, cost, budget, wl.k_cap, sel, kout, stream)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        step(*ev[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = t0.elapsed_time(t1) / steps
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    alg = sum(algorithmic_bytes(w.numel()) for w in weights)
+    k = int(kout.item())
+    kept = sorted(sel[:k].tolist())
+    kept_plain = sorted(sel_plain[:k_plain].tolist())
+    return {"value": wl.weight_bytes / (ms / 1e3) / 1e9, "unit": UNIT, "ms_per_step": ms,
+            "steps": steps,
+            "roofline": {"bound": "hbm", "achieved": alg / (kern_ms / 1e3) / 1e9, "peak": peak,
+                         "unit": "GB/s", "frac": alg / (kern_ms / 1e3) / 1e9 / peak,
+                         "kernel": "k_quant_score (AQNF4_SCORE_DQ_ABSMAX)"},
+            "selected": {"k": k, "of": L, "same_set_as_plain_score": kept == kept_plain}}
 
 
 def bench_workload(name, dev, stream, peak, steps):

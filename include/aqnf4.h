@@ -67,6 +67,16 @@ typedef enum {
 
 typedef enum { AQNF4_F16 = 0, AQNF4_BF16 = 1 } aqnf4_dtype;
 
+/* aqnf4_layer.flags bits. */
+enum {
+  /* Score the layer as NF4 + double quantization stores it ("QLoRA", "How It Works": the
+     quantization constants are quantized in turn): w_hat is rebuilt from the DQ constant
+     a'_b = fl(fl(code8_b / 255) * s) of its block, exactly what aqnf4_dequantize returns
+     from packed + codes8 + scales, instead of the binary32 absmax a_b.  The codes, packed
+     bytes, absmax, codes8 and scales written are the same either way. */
+  AQNF4_SCORE_DQ_ABSMAX = 1
+};
+
 /* One linear layer for aqnf4_layer_error.  All pointers are device pointers.
    w      : numel 16-bit weights, 16-byte aligned (required).
    packed : optional output, ceil(numel/2) bytes, 16-byte aligned.
@@ -78,7 +88,7 @@ typedef struct {
   const void* w;
   int64_t numel;
   int32_t dtype; /* aqnf4_dtype */
-  int32_t reserved; /* must be 0 */
+  int32_t flags; /* AQNF4_SCORE_* bits; other bits must be 0 */
   uint8_t* packed;
   float* absmax;
   uint8_t* codes8;
@@ -140,7 +150,8 @@ AQNF4_API size_t aqnf4_workspace_size(const aqnf4_layer* layers, int32_t num_lay
    reconstruction error), fused with NF4 quantization, packing and double quantization.
    layers: HOST array of num_layers descriptors (device pointers inside).  Each layer is
    quantized as in aqnf4_quantize; its optional outputs (packed, absmax, codes8 + scales)
-   are written; and, with w_hat = dtype_rn(fl(levels[code] * a_b)),
+   are written; and, with w_hat = dtype_rn(fl(levels[code] * a_b)) (a_b replaced by the
+   double-quantized a'_b for a layer flagged AQNF4_SCORE_DQ_ABSMAX),
      sq_err[l] = sum (x - w_hat)^2,  sq_w[l] = sum x^2,
      rel_err[l] = sqrt(sq_err[l] / sq_w[l])  (0 when sq_w[l] = 0; NaN after a NaN/inf input).
    The sums are taken in a fixed order, so repeated calls give identical bits.

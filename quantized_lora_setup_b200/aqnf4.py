@@ -27,6 +27,7 @@ AQNF4_ERR_WORKSPACE = 7
 
 AQNF4_F16 = 0
 AQNF4_BF16 = 1
+AQNF4_SCORE_DQ_ABSMAX = 1  # aqnf4_layer.flags
 
 _DT_CODE = {torch.float16: AQNF4_F16, torch.bfloat16: AQNF4_BF16}
 _CODE_DT = {AQNF4_F16: torch.float16, AQNF4_BF16: torch.bfloat16}
@@ -48,7 +49,7 @@ class aqnf4_layer(ctypes.Structure):
         ("w", ctypes.c_void_p),
         ("numel", ctypes.c_int64),
         ("dtype", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("flags", ctypes.c_int32),
         ("packed", ctypes.c_void_p),
         ("absmax", ctypes.c_void_p),
         ("codes8", ctypes.c_void_p),
@@ -166,14 +167,15 @@ def aqnf4_dequantize(packed: torch.Tensor, codes8: Optional[torch.Tensor],
 
 
 def make_layers(layers: Sequence[dict]):
-    """ctypes array of aqnf4_layer from dicts with keys w, packed, absmax, codes8, scales."""
+    """ctypes array of aqnf4_layer from dicts with keys w, packed, absmax, codes8, scales
+    and optionally flags (AQNF4_SCORE_* bits)."""
     arr = (aqnf4_layer * len(layers))()
     for i, d in enumerate(layers):
         w = d["w"]
         arr[i].w = w.data_ptr()
         arr[i].numel = w.numel()
         arr[i].dtype = dtype_code(w.dtype)
-        arr[i].reserved = 0
+        arr[i].flags = int(d.get("flags", 0))
         for key in ("packed", "absmax", "codes8", "scales"):
             t = d.get(key)
             setattr(arr[i], key, None if t is None else t.data_ptr())
@@ -288,13 +290,14 @@ class NF4Storage:
 
 
 def score_layers(weights: List[torch.Tensor], storages: Optional[List[NF4Storage]] = None,
-                 stream=None):
-    """Run the fused quantize+score pass: returns (sq_err f64[L], sq_w f64[L], rel_err f32[L])."""
+                 stream=None, dq_score: bool = False):
+    """Run the fused quantize+score pass: returns (sq_err f64[L], sq_w f64[L], rel_err f32[L]).
+    dq_score: score against the double-quantized constants (AQNF4_SCORE_DQ_ABSMAX)."""
     dev = weights[0].device
     L = len(weights)
     descs = []
     for i, w in enumerate(weights):
-        d = {"w": w}
+        d = {"w": w, "flags": AQNF4_SCORE_DQ_ABSMAX if dq_score else 0}
         if storages is not None:
             s = storages[i]
             d.update(packed=s.packed, codes8=s.codes8, scales=s.scales, absmax=s.absmax)

@@ -63,7 +63,8 @@ constexpr size_t kOutOff = kTileBytes;
 constexpr size_t kRedOff = kOutOff + kPackedTileBytes;
 constexpr size_t kRedBytes = 3 * kDqBlock * sizeof(float);
 constexpr size_t kMaxOff = kRedOff + kRedBytes;
-constexpr size_t kBarOff = kMaxOff + 16 * sizeof(float);
+constexpr size_t kPreOff = kMaxOff + 16 * sizeof(float);  // per-warp max for a DQ score
+constexpr size_t kBarOff = kPreOff + 16 * sizeof(float);
 constexpr size_t kSmemBytes = kBarOff + 16;
 
 struct LayerRec {
@@ -73,6 +74,8 @@ struct LayerRec {
   uint8_t* codes8;
   float* scales;
   int64_t numel;
+  int32_t flags;  // AQNF4_SCORE_* bits
+  int32_t pad;
 };
 
 struct QParams {
@@ -146,11 +149,13 @@ __device__ __forceinline__ void issue_tile(const QParams& p, int64_t tile, uint8
 }
 
 // Generic per-element path for a block whose absmax lies outside [2^-40, 2^40] (zero,
-// subnormal, huge or not finite).  Re-reads the block (natural element order) from shared memory, rewrites
-// this thread's packed words and returns the normalised sums (err, w^2) -- scaled by a^2
-// later like the fast path's.
+// subnormal, huge or not finite).  Re-reads the block (natural element order) from shared
+// memory, rewrites this thread's packed words and returns the normalised sums (err, w^2) --
+// scaled by a^2 later like the fast path's.  ar is the constant w_hat is rebuilt from: a,
+// or the double-quantized a' (at most ~2a, so the normalised terms stay small).
 template <int DT, bool SCORE>
-__device__ __noinline__ float2 block_generic(const uint8_t* my, float a, const QParams& p,
+__device__ __noinline__ float2 block_generic(const uint8_t* my, float a, float ar,
+                                             const QParams& p,
                                              uint8_t* ost) {  // ost: this block's 32 bytes
   using F = Fmt<DT>;
   const bool zero = (a == 0.0f);
@@ -177,7 +182,7 @@ __device__ __noinline__ float2 block_generic(const uint8_t* my, float a, const Q
       }
       pk |= static_cast<uint32_t>(code) << ((i >> 1) * 8 + ((i & 1) ? 0 : 4));
       if (SCORE && !zero) {
-        const float wh = F::round_trip(__fmul_rn(p.level[code], a));
+        const float wh = F::round_trip(__fmul_rn(p.level[code], ar));
         const float d = __fmul_rn(__fsub_rn(__fmul_rn(x, scale), __fmul_rn(wh, scale)), r);
         se = __fmaf_rn(d, d, se);
         sw = __fmaf_rn(v, v, sw);
@@ -200,6 +205,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   uint8_t* stage = smem;
   float* red = reinterpret_cast<float*>(smem + kRedOff);   // [3 = err, w2, scale][256]
   float* wmax = reinterpret_cast<float*>(smem + kMaxOff);  // [kWarps]
+  uint32_t* wpre = reinterpret_cast<uint32_t*>(smem + kPreOff);  // [kWarps]
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kBarOff);
   int* abort_flag = reinterpret_cast<int*>(smem + kBarOff + 8);
   const uint32_t bar_a = smem_addr(bar);
@@ -264,6 +270,29 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       r[b] = fast[b] ? __frcp_rn(a[b]) : 0.0f;
     }
 
+    // ---- the constant w_hat is rebuilt from: a, or for a DQ score the double-quantized
+    // a' = fl(fl(code8/255) s) with s the tile's (DQ block's) maximum.  a' <= ~2a (code8 > 0
+    // needs a >= s/510), so the fast path's range argument still holds.  The branch is
+    // uniform over the CTA (one layer per tile).
+    float ar[kBpt];
+#pragma unroll
+    for (int b = 0; b < kBpt; ++b) ar[b] = a[b];
+    if (SCORE && (L.flags & AQNF4_SCORE_DQ_ABSMAX)) {
+      uint32_t m = 0;
+#pragma unroll
+      for (int b = 0; b < kBpt; ++b)
+        if (t + b * kThreads < nblk) m = max(m, __float_as_uint(a[b]));
+      m = __reduce_max_sync(kFull, m);
+      if (lane == 0) wpre[warp] = m;
+      __syncthreads();
+      uint32_t sb = 0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) sb = max(sb, wpre[w]);
+      const float s = __uint_as_float(sb);
+#pragma unroll
+      for (int b = 0; b < kBpt; ++b) ar[b] = dq_constant(dq_code(a[b], s), s);
+    }
+
     // ---- pass 2: codes, packing, error; the blocks' chains interleave (all lanes run this
     // so the shuffles stay converged)
     f32x2 es2[kBpt], ws2[kBpt], r2[kBpt], a2[kBpt];
@@ -271,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     for (int b = 0; b < kBpt; ++b) {
       es2[b] = ws2[b] = pair(0.0f, 0.0f);
       r2[b] = pair(r[b], r[b]);
-      a2[b] = pair(a[b], a[b]);
+      a2[b] = pair(ar[b], ar[b]);
     }
     const f32x2 ca2 = pair(p.curve_a, p.curve_a), cb2 = pair(p.curve_b, p.curve_b);
     const f32x2 off2 = pair(8388616.0f, 8388616.0f);  // 2^23 + 8
@@ -335,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       // factor that turns this block's sums into weight units once squared
       float sum_scale = 1.0f;
       if (!fast[b]) {
-        sums = block_generic<DT, SCORE>(stage + blk * 128, a[b], p, ost + blk * 32);
+        sums = block_generic<DT, SCORE>(stage + blk * 128, a[b], ar[b], p, ost + blk * 32);
         sum_scale = a[b];
       }
       if (SCORE) {
@@ -495,7 +524,7 @@ void fill_tables(QParams& p, const Tables& tb) {
 }
 
 aqnf4_status check_layer(const aqnf4_layer& L) {
-  if (!L.w || L.numel < 1 || L.reserved != 0) return AQNF4_ERR_INVALID_ARG;
+  if (!L.w || L.numel < 1 || (L.flags & ~AQNF4_SCORE_DQ_ABSMAX) != 0) return AQNF4_ERR_INVALID_ARG;
   if (!valid_dtype(L.dtype)) return AQNF4_ERR_DTYPE;
   if (L.codes8 && !L.scales) return AQNF4_ERR_INVALID_ARG;
   if (!is_aligned(L.w, 16) || !is_aligned(L.packed, 16) || !is_aligned(L.absmax, 4) ||
@@ -555,7 +584,7 @@ aqnf4_status aqnf4_quantize(const void* w, int32_t dtype, int64_t n, uint8_t* pa
   fill_tables(p, *tb);
   p.tile_begin[0] = 0;
   p.tile_begin[1] = static_cast<int32_t>(p.num_tiles);
-  p.layers[0] = LayerRec{w, packed, absmax, nullptr, nullptr, n};
+  p.layers[0] = LayerRec{w, packed, absmax, nullptr, nullptr, n, 0, 0};
   if (p.num_tiles > INT32_MAX) return AQNF4_ERR_INVALID_ARG;
   return launch_main_dt(dtype, false, p, stream) == cudaSuccess ? AQNF4_OK : AQNF4_ERR_CUDA;
 }
@@ -598,7 +627,7 @@ aqnf4_status aqnf4_layer_error(const aqnf4_layer* layers, int32_t num_layers, vo
       if (tiles + lt > INT32_MAX) break;
       p.tile_begin[n] = static_cast<int32_t>(tiles);
       f.tile_begin[n] = static_cast<int32_t>(tiles);
-      p.layers[n] = LayerRec{L.w, L.packed, L.absmax, L.codes8, L.scales, L.numel};
+      p.layers[n] = LayerRec{L.w, L.packed, L.absmax, L.codes8, L.scales, L.numel, L.flags, 0};
       tiles += lt;
       ++n;
     }

@@ -77,7 +77,7 @@ class FakeTensor:
 
 def layer(addr=0x10000, numel=100, dtype=aqnf4.AQNF4_BF16, **kw):
     d = aqnf4.aqnf4_layer()
-    d.w, d.numel, d.dtype, d.reserved = addr, numel, dtype, kw.get("reserved", 0)
+    d.w, d.numel, d.dtype, d.flags = addr, numel, dtype, kw.get("flags", 0)
     d.packed = kw.get("packed")
     d.absmax = kw.get("absmax")
     d.codes8 = kw.get("codes8")
@@ -115,8 +115,10 @@ def test_argument_checks_return_before_any_launch(lib):
     one = (aqnf4.aqnf4_layer * 1)(layer())
     ws = V(0x100000)
     assert lib.aqnf4_layer_error(one, 0, ws, 4096, None, None, None, None, None) == aqnf4.AQNF4_ERR_INVALID_ARG
-    bad = (aqnf4.aqnf4_layer * 1)(layer(reserved=1))
-    assert lib.aqnf4_layer_error(bad, 1, ws, 4096, None, None, None, None, None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    for flags in (2, 4, -1):  # only AQNF4_SCORE_DQ_ABSMAX is defined
+        bad = (aqnf4.aqnf4_layer * 1)(layer(flags=flags))
+        assert lib.aqnf4_layer_error(bad, 1, ws, 4096, None, None, None, None, None) == \
+            aqnf4.AQNF4_ERR_INVALID_ARG
     bad = (aqnf4.aqnf4_layer * 1)(layer(codes8=0x5000))
     assert lib.aqnf4_layer_error(bad, 1, ws, 4096, None, None, None, None, None) == aqnf4.AQNF4_ERR_INVALID_ARG
     bad = (aqnf4.aqnf4_layer * 1)(layer(dtype=9))

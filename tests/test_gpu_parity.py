@@ -347,3 +347,81 @@ def test_quantize_exact_midpoint_ties(cuda):
     ose, osw, orel = oracle.layer_error(bits(w), DT[dt])
     assert se.item() == pytest.approx(ose, rel=RTOL)
     assert rel.item() == pytest.approx(orel, rel=RTOL)
+
+
+# ------------------------------------------------- score against the DQ constants
+
+
+def _dq_case_layers():
+    """Ragged random layers of both formats plus one with special blocks inside a DQ block:
+    zeros, a block far below the DQ block's maximum (its constant double-quantizes to 0),
+    a subnormal maximum and a huge one."""
+    rng = np.random.default_rng(31)
+    out = []
+    for n, dt in ((1, torch.bfloat16), (65, torch.float16), (16385, torch.bfloat16),
+                  (3 * 16384 + 17, torch.float16), (100003, torch.bfloat16)):
+        sig = np.repeat(rng.uniform(0.002, 0.05, n // 64 + 1), 64)[:n]
+        out.append(torch.from_numpy((rng.standard_normal(n) * sig).astype(np.float32)).to(dt))
+    blocks = [rng.standard_normal(64) * 0.02 for _ in range(300)]
+    blocks[3] = np.zeros(64)
+    blocks[4] = rng.standard_normal(64) * 1e-6           # code8 0: rebuilt from a' = 0
+    blocks[5] = rng.standard_normal(64) * 1e-39          # subnormal absmax (generic path)
+    blocks[6] = rng.standard_normal(64) * 3e20           # above 2^40 (generic path)
+    blocks[7] = rng.standard_normal(64) * 2e-4           # small non-zero code8
+    out.append(torch.from_numpy(np.concatenate(blocks).astype(np.float32)).to(torch.bfloat16))
+    return out
+
+
+def test_dq_score_matches_oracle_and_keeps_the_storage(cuda):
+    ws = _dq_case_layers()
+    dev = [w.to(cuda) for w in ws]
+    plain_st = [aqnf4.NF4Storage(w.numel(), cuda) for w in dev]
+    dq_st = [aqnf4.NF4Storage(w.numel(), cuda) for w in dev]
+    _, _, _ = aqnf4.score_layers(dev, plain_st)
+    se, sw, rel = aqnf4.score_layers(dev, dq_st, dq_score=True)
+    torch.cuda.synchronize()
+    for i, w in enumerate(ws):
+        ose, osw, orel = oracle.layer_error_dq(bits(w), DT[w.dtype])
+        assert se[i].item() == pytest.approx(ose, rel=RTOL), i
+        assert sw[i].item() == pytest.approx(osw, rel=RTOL), i
+        assert rel[i].item() == pytest.approx(orel, rel=RTOL), i
+        for name in ("packed", "codes8", "scales"):  # the flag changes only the score
+            assert torch.equal(getattr(dq_st[i], name), getattr(plain_st[i], name)), (i, name)
+
+
+def test_dq_and_plain_scores_in_one_call(cuda):
+    """Flags are per layer: alternating layers in one launch each get their own score."""
+    ws = _dq_case_layers()
+    dev = [w.to(cuda) for w in ws]
+    descs = aqnf4.make_layers([{"w": w, "flags": aqnf4.AQNF4_SCORE_DQ_ABSMAX if i % 2 else 0}
+                               for i, w in enumerate(dev)])
+    L = len(dev)
+    wsp = torch.empty(max(256, aqnf4.aqnf4_workspace_size(descs)), dtype=torch.uint8, device=cuda)
+    se = torch.empty(L, dtype=torch.float64, device=cuda)
+    sw = torch.empty(L, dtype=torch.float64, device=cuda)
+    rel = torch.empty(L, dtype=torch.float32, device=cuda)
+    aqnf4.aqnf4_layer_error(descs, wsp, se, sw, rel)
+    torch.cuda.synchronize()
+    for i, w in enumerate(ws):
+        ref = oracle.layer_error_dq if i % 2 else oracle.layer_error
+        ose, _, orel = ref(bits(w), DT[w.dtype])
+        assert se[i].item() == pytest.approx(ose, rel=RTOL), i
+        assert rel[i].item() == pytest.approx(orel, rel=RTOL), i
+
+
+def test_dq_score_nonfinite_tile_is_nan(cuda):
+    """An infinite weight makes its DQ block's scale infinite, so every constant of that
+    block rebuilds as NaN: the score is NaN (as in the oracle) and the flag is set."""
+    rng = np.random.default_rng(32)
+    z = rng.standard_normal(64 * 300) * 0.02
+    z[64 * 10 + 3] = np.inf
+    w = torch.from_numpy(z.astype(np.float32)).to(torch.bfloat16)
+    flag = torch.zeros(1, dtype=torch.int32, device=cuda)
+    descs = aqnf4.make_layers([{"w": w.to(cuda), "flags": aqnf4.AQNF4_SCORE_DQ_ABSMAX}])
+    wsp = torch.empty(256, dtype=torch.uint8, device=cuda)
+    rel = torch.empty(1, dtype=torch.float32, device=cuda)
+    aqnf4.aqnf4_layer_error(descs, wsp, None, None, rel, flag)
+    torch.cuda.synchronize()
+    assert math.isnan(oracle.layer_error_dq(bits(w), oracle.BF16)[2])
+    assert math.isnan(rel.item())
+    assert flag.item() == aqnf4.AQNF4_ERR_NONFINITE

@@ -58,7 +58,7 @@ def test_noalloc_rejects_requests_above_its_scratch():
     """More than 2^19 tiles of 16384 elements is refused before anything is launched."""
     lib = aqnf4.library()
     d = aqnf4.aqnf4_layer()
-    d.w, d.numel, d.dtype, d.reserved = 0x10000, (1 << 19) * 16384 + 1, aqnf4.AQNF4_BF16, 0
+    d.w, d.numel, d.dtype, d.flags = 0x10000, (1 << 19) * 16384 + 1, aqnf4.AQNF4_BF16, 0
     arr = (aqnf4.aqnf4_layer * 1)(d)
     before = lib.aqnf4_launch_count()
     st = lib.aqnf4_layer_error_noalloc(arr, 1, None, None, None, None, None)
