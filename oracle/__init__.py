@@ -37,6 +37,9 @@ def load():
     lib.oracle_layer_error.restype = None
     lib.oracle_layer_error_dq.argtypes = [P, ctypes.c_int, i64, P, P, P, P, P]
     lib.oracle_layer_error_dq.restype = ctypes.c_int
+    lib.oracle_select_blocks.argtypes = [P, P, P, P, ctypes.c_int, ctypes.c_int, i64,
+                                         ctypes.c_int, P, P, P]
+    lib.oracle_select_blocks.restype = ctypes.c_int
     lib.oracle_double_quant.argtypes = [P, i64, P, P, P]
     lib.oracle_double_quant.restype = None
     lib.oracle_dequantize.argtypes = [P, P, P, P, i64, ctypes.c_int, P, P]
@@ -163,6 +166,26 @@ def select_topk(rel_err, cost, budget: int, k_cap: int = -1):
     return [int(i) for i in sel[: k[0]]]
 
 
+BLOCKS_BY_DEPTH = 0
+BLOCKS_BY_ERROR = 1
+
+
+def select_blocks(sq_err, sq_w, block_of, cost, num_blocks: int, budget: int, order: int):
+    """(ranking list[int], block scores float32[B], kept k) of the block-level selection."""
+    se = np.ascontiguousarray(sq_err, np.float64)
+    sw = np.ascontiguousarray(sq_w, np.float64)
+    bo = np.ascontiguousarray(block_of, np.int32)
+    c = np.ascontiguousarray(cost, np.int64)
+    rank = np.zeros(max(num_blocks, 1), np.int32)
+    err = np.zeros(max(num_blocks, 1), np.float32)
+    k = np.zeros(1, np.int32)
+    if load().oracle_select_blocks(_ptr(se), _ptr(sw), _ptr(bo), _ptr(c), se.size, num_blocks,
+                                   int(budget), int(order), _ptr(rank), _ptr(err),
+                                   _ptr(k)) != 0:
+        raise ValueError("invalid block selection arguments")
+    return [int(i) for i in rank[:num_blocks]], err[:num_blocks].copy(), int(k[0])
+
+
 def f32_to_dtype_bits(values, dtype):
     lib = load()
     v = np.asarray(values, np.float32).reshape(-1)
@@ -176,7 +199,7 @@ def dtype_bits_to_f32(bits, dtype):
 
 
 __all__ = ["F16", "BF16", "load", "default_pmax", "codebook", "quantize", "layer_error",
-           "layer_error_dq",
+           "layer_error_dq", "select_blocks", "BLOCKS_BY_DEPTH", "BLOCKS_BY_ERROR",
            "double_quant", "dequantize", "cost_bytes", "select_topk", "f32_to_dtype_bits",
            "dtype_bits_to_f32"]
 

@@ -452,6 +452,54 @@ int oracle_select_topk(const float* e, const int64_t* cost, int L, int64_t budge
   return 0;
 }
 
+/* Block-level selection for the speed setting ([AQLoRA/abs]: a speed setting adapts only
+   the top blocks, so the backward pass stops early; [AQLoRA/TD]: it promotes only the top
+   blocks).  Each layer l belongs to transformer block block_of[l] in [0, B).  A block costs
+   the sum of its layers' costs.  Its score is the relative error of all its layers together,
+   sqrt(sum sq_err / sum sq_w) with the sums in binary64 in layer order (0 when the block's
+   sum sq_w is 0).  order 0 ranks the blocks by depth, last block first: the plain reading
+   of "top blocks".  order 1 ranks them by score (desc, NaN last, index asc).  The kept
+   blocks are the longest prefix of the ranking whose total cost fits the budget.  rank[B]
+   receives the whole ranking, block_err[B] the scores and *k_out the number kept.
+   Returns 0, or -1 for invalid arguments. */
+int oracle_select_blocks(const double* sq_err, const double* sq_w, const int* block_of,
+                         const int64_t* cost, int L, int B, int64_t budget, int order,
+                         int* rank, float* block_err, int* k_out) {
+  if (L < 0 || B < 1 || budget < 0 || (order != 0 && order != 1)) return -1;
+  for (int l = 0; l < L; ++l)
+    if (block_of[l] < 0 || block_of[l] >= B) return -1;
+  int64_t bcost[B];
+  for (int b = 0; b < B; ++b) {
+    double se = 0.0, sw = 0.0;
+    bcost[b] = 0;
+    for (int l = 0; l < L; ++l) {
+      if (block_of[l] != b) continue;
+      se += sq_err[l];
+      sw += sq_w[l];
+      bcost[b] += cost[l];
+    }
+    double e = sw == 0.0 ? 0.0 : sqrt(se / sw);
+    if (isnan(se) || isnan(sw)) e = NAN;
+    block_err[b] = (float)e;
+  }
+  for (int i = 0; i < B; ++i) rank[i] = order == 0 ? B - 1 - i : i;
+  if (order == 1) {
+    for (int a = 0; a < B; ++a) {
+      int best = a;
+      for (int c = a + 1; c < B; ++c)
+        if (or_before(block_err, rank[c], rank[best])) best = c;
+      int t = rank[a];
+      rank[a] = rank[best];
+      rank[best] = t;
+    }
+  }
+  int64_t used = 0;
+  int k = 0;
+  while (k < B && used + bcost[rank[k]] <= budget) used += bcost[rank[k++]];
+  *k_out = k;
+  return 0;
+}
+
 /* bit helpers exported for the tests' conversion pins */
 uint16_t oracle_f32_to_dtype_bits(float f, int dtype) { return or_round_to_dtype(f, dtype); }
 float oracle_dtype_bits_to_f32(uint16_t h, int dtype) { return or_load(h, dtype); }

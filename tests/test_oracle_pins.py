@@ -477,6 +477,81 @@ def test_select_rules():
         oracle.select_topk(e, [1] * 5, -1)
 
 
+# ------------------------------------------------------ block-level selection
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_blocks_of_one_layer_select_like_layers(seed):
+    """With one layer per block, ranking blocks by error is the layer selection itself."""
+    rng = np.random.default_rng(seed)
+    L = 12
+    sw = rng.uniform(0.5, 50.0, L)
+    rel = rng.uniform(0.05, 0.2, L).astype(np.float32)
+    rel[3] = rel[7]                                   # a tie: lower index first
+    se = (rel.astype(np.float64) ** 2) * sw
+    # the block score rounds sqrt(se/sw) to binary32: use exactly what the layers report
+    rel = np.sqrt(se / sw).astype(np.float32)
+    cost = rng.integers(1, 100, L)
+    for budget in (0, 50, 200, 400, 10 ** 6):
+        rank, err, k = oracle.select_blocks(se, sw, np.arange(L), cost, L, budget,
+                                            oracle.BLOCKS_BY_ERROR)
+        assert np.array_equal(err.view(np.uint32), rel.view(np.uint32))
+        assert rank[:k] == oracle.select_topk(rel, cost, budget)
+
+
+def test_block_score_closed_forms():
+    """A block whose layers share one relative error e scores e; in general the block score
+    lies between its layers' smallest and largest relative errors."""
+    rng = np.random.default_rng(5)
+    block_of = np.repeat(np.arange(4), 7)
+    sw = rng.uniform(1.0, 30.0, block_of.size)
+    rel = rng.uniform(0.05, 0.2, block_of.size)
+    rel[block_of == 2] = 0.125                        # exact in binary and in its square
+    se = rel ** 2 * sw
+    _, err, _ = oracle.select_blocks(se, sw, block_of, np.ones(block_of.size), 4, 0,
+                                     oracle.BLOCKS_BY_ERROR)
+    assert err[2] == np.float32(0.125)
+    for b in range(4):
+        r = rel[block_of == b]
+        assert r.min() * (1 - 1e-6) <= err[b] <= r.max() * (1 + 1e-6)
+
+
+def test_blocks_by_depth_keep_the_top_that_fits():
+    """By depth, the kept blocks are the last k blocks for the largest k whose summed cost
+    fits (brute force over k); a block with no layers costs nothing."""
+    rng = np.random.default_rng(6)
+    B = 9
+    block_of = np.sort(rng.integers(0, B, 40))
+    block_of[block_of == 4] = 5                       # block 4 has no layers
+    cost = rng.integers(1, 50, block_of.size)
+    se = rng.uniform(0, 1, block_of.size)
+    sw = rng.uniform(1, 2, block_of.size)
+    bcost = np.array([cost[block_of == b].sum() for b in range(B)])
+    for budget in range(0, int(bcost.sum()) + 5, 7):
+        rank, _, k = oracle.select_blocks(se, sw, block_of, cost, B, budget,
+                                          oracle.BLOCKS_BY_DEPTH)
+        assert rank == list(range(B - 1, -1, -1))
+        best = 0
+        for kk in range(B + 1):
+            if bcost[B - kk:].sum() <= budget:
+                best = kk
+            else:
+                break
+        assert k == best
+
+
+def test_block_selection_nan_last_and_argument_checks():
+    se = np.array([0.1, np.nan, 0.4, 0.2])
+    sw = np.ones(4)
+    rank, err, k = oracle.select_blocks(se, sw, [0, 1, 2, 3], [1, 1, 1, 1], 4, 10,
+                                        oracle.BLOCKS_BY_ERROR)
+    assert rank == [2, 3, 0, 1] and k == 4 and np.isnan(err[1])
+    with pytest.raises(ValueError):
+        oracle.select_blocks(se, sw, [0, 1, 2, 4], [1, 1, 1, 1], 4, 10, oracle.BLOCKS_BY_ERROR)
+    with pytest.raises(ValueError):
+        oracle.select_blocks(se, sw, [0, 1, 2, 3], [1, 1, 1, 1], 4, -1, oracle.BLOCKS_BY_DEPTH)
+
+
 def test_cost_bytes_closed_form():
     for n in (1, 7, 64, 65, 4096 * 4096, 11008 * 4096, 16385):
         nb = -(-n // 64)
