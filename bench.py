@@ -367,6 +367,9 @@ def run_native(args):
     if not args.no_dequant:
         result["dequant"] = bench_dequant(dev, stream, peak)
 
+    if world == 1:
+        result["select_blocks"] = bench_select_blocks(wl, se, sw, cost, budget, dev, stream)
+
     if world == 1 and not args.no_dq_score:
         result["dq_score"] = bench_dq_score(weights, stor, wl, cost, budget, sel, k_sel, dev,
                                             stream, peak, steps=min(K, 100))
@@ -401,6 +404,37 @@ def run_native(args):
     if rank == 0:
         print(json.dumps(result), flush=True)
     return 0
+
+
+def bench_select_blocks(wl, se, sw, cost, budget, dev, stream, reps=200):
+    """Block-level selection (speed setting) on the step's scores, both orders: the blocks
+    kept under the budget, the lowest kept block, and the kernel's time per launch."""
+    import torch
+
+    from quantized_lora_setup_b200 import aqnf4, synth
+    block_of = torch.tensor(synth.block_index(wl), dtype=torch.int32, device=dev)
+    B = int(block_of.max().item()) + 1
+    out = {"blocks": B}
+    for name, order in (("by_depth", aqnf4.AQNF4_BLOCKS_BY_DEPTH),
+                        ("by_error", aqnf4.AQNF4_BLOCKS_BY_ERROR)):
+        rank = torch.empty(B, dtype=torch.int32, device=dev)
+        k = torch.empty(1, dtype=torch.int32, device=dev)
+
+        def run():
+            aqnf4.aqnf4_select_blocks(se, sw, block_of, cost, B, budget, order, rank, None, k,
+                                      stream)
+        for _ in range(3):
+            run()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(reps):
+            run()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        kept = rank[: int(k.item())].tolist()
+        out[name] = {"kept": kept, "lowest_kept_block": min(kept) if kept else None,
+                     "us_per_launch": t0.elapsed_time(t1) * 1e3 / reps}
+    return out
 
 
 def bench_dq_score(weights, stor, wl, cost, budget, sel_plain, k_plain, dev, stream, peak, steps):

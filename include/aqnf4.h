@@ -206,6 +206,33 @@ AQNF4_API aqnf4_status aqnf4_selftest_wait_timeout(int64_t timeout_ns, int32_t* 
    read as a budget on this quantity.) */
 AQNF4_API int64_t aqnf4_cost_bytes(int64_t n);
 
+/* Block-level selection for the speed setting (arxivdaily 2608.23816, "English abstract":
+   a speed setting adapts only the top blocks, so the backward pass stops early; "AQLoRA:
+   ...", "Technical Details": it promotes only the top blocks).  Layer l belongs to
+   transformer block block_of[l] in [0, num_blocks).  A block costs the sum of its layers'
+   cost_bytes.  Its score block_err is the relative error of its layers together,
+   sqrt(sum sq_err / sum sq_w), summed in binary64 in layer order (0 when sum sq_w = 0; NaN
+   after a NaN input).  order AQNF4_BLOCKS_BY_DEPTH ranks the blocks from the last one down
+   (the pages' "top blocks"; the lowest kept block is where the backward pass can stop);
+   AQNF4_BLOCKS_BY_ERROR ranks them by block_err descending (equal scores: lower index
+   first; NaN last).  The kept blocks are the longest prefix of the ranking whose summed
+   cost is within budget_bytes.
+   sq_err, sq_w (device double[num_layers], e.g. aqnf4_layer_error's outputs), block_of
+   (device int32[num_layers]) and cost_bytes (device int64[num_layers]) are inputs;
+   block_rank (device int32[num_blocks]) receives the whole ranking, block_err (optional,
+   device float[num_blocks]) the scores and k_out (device int32[1]) the number of blocks kept,
+   or -1 when a block_of entry lies outside [0, num_blocks) (the other outputs are then
+   meaningless).  1 <= num_blocks <= 2048.  One thread block.
+   Errors: INVALID_ARG (NULL pointer, a size out of range, budget_bytes < 0, unknown order),
+   ALIGNMENT, CUDA. */
+enum { AQNF4_BLOCKS_BY_DEPTH = 0, AQNF4_BLOCKS_BY_ERROR = 1 };
+AQNF4_API aqnf4_status aqnf4_select_blocks(const double* sq_err, const double* sq_w,
+                                           const int32_t* block_of, const int64_t* cost_bytes,
+                                           int32_t num_layers, int32_t num_blocks,
+                                           int64_t budget_bytes, int32_t order,
+                                           int32_t* block_rank, float* block_err,
+                                           int32_t* k_out, cudaStream_t stream);
+
 /* The fused pass's code lookup, for inspection (host only; no counterpart on the pages,
    which define the code as the nearest level, i.e. the number of midpoints below v).
    curve[2] = (a, b); slot_mid[32], slot_level[32].  For a normalised value v with

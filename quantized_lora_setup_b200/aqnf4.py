@@ -28,6 +28,8 @@ AQNF4_ERR_WORKSPACE = 7
 AQNF4_F16 = 0
 AQNF4_BF16 = 1
 AQNF4_SCORE_DQ_ABSMAX = 1  # aqnf4_layer.flags
+AQNF4_BLOCKS_BY_DEPTH = 0  # aqnf4_select_blocks orders
+AQNF4_BLOCKS_BY_ERROR = 1
 
 _DT_CODE = {torch.float16: AQNF4_F16, torch.bfloat16: AQNF4_BF16}
 _CODE_DT = {AQNF4_F16: torch.float16, AQNF4_BF16: torch.bfloat16}
@@ -92,6 +94,8 @@ def library() -> ctypes.CDLL:
     lib.aqnf4_select_topk.restype = st
     lib.aqnf4_selftest_wait_timeout.argtypes = [i64, P, P, P]
     lib.aqnf4_selftest_wait_timeout.restype = st
+    lib.aqnf4_select_blocks.argtypes = [P, P, P, P, i32, i32, i64, i32, P, P, P, P]
+    lib.aqnf4_select_blocks.restype = st
     lib.aqnf4_slot_tables.argtypes = [P, P, P]
     lib.aqnf4_slot_tables.restype = st
     lib.aqnf4_cost_bytes.argtypes = [i64]
@@ -219,6 +223,16 @@ def aqnf4_selftest_wait_timeout(timeout_ns: int, dev_flag: torch.Tensor,
                                 waited_ns: Optional[torch.Tensor] = None, stream=None) -> None:
     _check(library().aqnf4_selftest_wait_timeout(int(timeout_ns), _ptr(dev_flag), _ptr(waited_ns),
                                                  _stream(stream)), "aqnf4_selftest_wait_timeout")
+
+
+def aqnf4_select_blocks(sq_err: torch.Tensor, sq_w: torch.Tensor, block_of: torch.Tensor,
+                        cost_bytes: torch.Tensor, num_blocks: int, budget_bytes: int, order: int,
+                        block_rank: torch.Tensor, block_err: Optional[torch.Tensor],
+                        k_out: torch.Tensor, stream=None) -> None:
+    _check(library().aqnf4_select_blocks(_ptr(sq_err), _ptr(sq_w), _ptr(block_of),
+                                         _ptr(cost_bytes), sq_err.numel(), num_blocks,
+                                         budget_bytes, order, _ptr(block_rank), _ptr(block_err),
+                                         _ptr(k_out), _stream(stream)), "aqnf4_select_blocks")
 
 
 def aqnf4_slot_tables():

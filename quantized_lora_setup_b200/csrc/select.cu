@@ -1,4 +1,5 @@
-// select.cu -- top-K layers under a byte budget (aqnf4_select_topk).
+// select.cu -- top-K layers under a byte budget (aqnf4_select_topk) and the block-level
+// selection of the speed setting (aqnf4_select_blocks).
 //
 // arxivdaily 2608.23816, "English abstract": the pass ranks layers by NF4 reconstruction
 // error and keeps the top-K in fp16 under a memory budget; "AQLoRA: A Zero-Search Recipe
@@ -81,6 +82,59 @@ __global__ void __launch_bounds__(kSelThreads) k_select_topk(const float* __rest
   if (t == 0) *k_out = first_out;
 }
 
+// Block-level selection ("English abstract": a speed setting adapts only the top blocks, so
+// the backward pass stops early).  One CTA: each thread owns blocks b = t, t + 1024, ... and
+// sums its layers in layer order in binary64 (the same order as any other caller, so the
+// scores are reproducible to the bit); the ranking is the count of blocks ranked before
+// each block; one thread then walks the ranking against the budget.
+constexpr int kMaxBlocks = 2048;
+
+__global__ void __launch_bounds__(kSelThreads) k_select_blocks(
+    const double* __restrict__ sq_err, const double* __restrict__ sq_w,
+    const int32_t* __restrict__ block_of, const int64_t* __restrict__ cost, int L, int B,
+    int64_t budget, int order, int32_t* block_rank, float* block_err, int32_t* k_out) {
+  __shared__ float s_err[kMaxBlocks];
+  __shared__ int64_t s_cost[kMaxBlocks];
+  __shared__ int bad;
+  const int t = threadIdx.x;
+  if (t == 0) bad = 0;
+  __syncthreads();
+  for (int b = t; b < B; b += kSelThreads) {
+    double se = 0.0, sw = 0.0;
+    int64_t c = 0;
+    for (int l = 0; l < L; ++l) {
+      const int32_t bl = __ldg(block_of + l);
+      if (bl < 0 || bl >= B) bad = 1;
+      if (bl != b) continue;
+      se += __ldg(sq_err + l);
+      sw += __ldg(sq_w + l);
+      c += __ldg(cost + l);
+    }
+    double e = sw == 0.0 ? 0.0 : sqrt(se / sw);
+    if (se != se || sw != sw) e = __longlong_as_double(0x7ff8000000000000ll);
+    s_err[b] = __double2float_rn(e);
+    s_cost[b] = c;
+    if (block_err) block_err[b] = s_err[b];
+  }
+  __syncthreads();
+  for (int b = t; b < B; b += kSelThreads) {
+    int rank = B - 1 - b;  // by depth: the last block first
+    if (order == 1) {
+      rank = 0;
+      for (int j = 0; j < B; ++j) rank += ranks_before(s_err[j], j, s_err[b], b) ? 1 : 0;
+    }
+    block_rank[rank] = b;
+  }
+  __syncthreads();
+  if (t == 0) {
+    int64_t used = 0;
+    int k = 0;
+    while (k < B && used + s_cost[__ldcg(block_rank + k)] <= budget)
+      used += s_cost[__ldcg(block_rank + k++)];
+    *k_out = bad ? -1 : k;
+  }
+}
+
 }  // namespace
 }  // namespace aqnf4
 
@@ -96,6 +150,27 @@ extern "C" aqnf4_status aqnf4_select_topk(const float* rel_err, const int64_t* c
     return AQNF4_ERR_ALIGNMENT;
   k_select_topk<<<1, kSelThreads, 0, stream>>>(rel_err, cost_bytes, L, budget_bytes, k_cap,
                                                sel_idx, k_out);
+  count_launches(1);
+  return cudaGetLastError() == cudaSuccess ? AQNF4_OK : AQNF4_ERR_CUDA;
+}
+
+extern "C" aqnf4_status aqnf4_select_blocks(const double* sq_err, const double* sq_w,
+                                            const int32_t* block_of, const int64_t* cost_bytes,
+                                            int32_t num_layers, int32_t num_blocks,
+                                            int64_t budget_bytes, int32_t order,
+                                            int32_t* block_rank, float* block_err,
+                                            int32_t* k_out, cudaStream_t stream) {
+  if (!sq_err || !sq_w || !block_of || !cost_bytes || !block_rank || !k_out ||
+      num_layers < 1 || num_blocks < 1 || num_blocks > kMaxBlocks || budget_bytes < 0 ||
+      (order != AQNF4_BLOCKS_BY_DEPTH && order != AQNF4_BLOCKS_BY_ERROR))
+    return AQNF4_ERR_INVALID_ARG;
+  if (!is_aligned(sq_err, 8) || !is_aligned(sq_w, 8) || !is_aligned(block_of, 4) ||
+      !is_aligned(cost_bytes, 8) || !is_aligned(block_rank, 4) || !is_aligned(block_err, 4) ||
+      !is_aligned(k_out, 4))
+    return AQNF4_ERR_ALIGNMENT;
+  k_select_blocks<<<1, kSelThreads, 0, stream>>>(sq_err, sq_w, block_of, cost_bytes, num_layers,
+                                                 num_blocks, budget_bytes, order, block_rank,
+                                                 block_err, k_out);
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? AQNF4_OK : AQNF4_ERR_CUDA;
 }

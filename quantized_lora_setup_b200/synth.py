@@ -25,7 +25,7 @@ normal draws.  Layer ``l`` of a workload with seed ``s`` uses the stream
 bytes one side saw to the other.
 """
 from dataclasses import dataclass
-from typing import Tuple
+from typing import List, Tuple
 
 import numpy as np
 import torch
@@ -69,6 +69,11 @@ class Workload:
 
 def _blocks(prefix_shapes, nblocks):
     return [(f"blk{b}.{n}", r, c) for b in range(nblocks) for (n, r, c) in prefix_shapes]
+
+
+def block_index(wl: Workload) -> List[int]:
+    """Transformer block of every layer ("blk<b>.<name>"), for the block-level selection."""
+    return [int(l.name.split(".", 1)[0][3:]) for l in wl.layers]
 
 
 def tiny(seed: int = 0) -> Workload:
@@ -196,6 +201,6 @@ def bits_u16(t: torch.Tensor) -> np.ndarray:
     return t.view(torch.int16).numpy().view(np.uint16)
 
 
-__all__ = ["GIB", "LayerSpec", "Workload", "tiny", "model_1p4b", "model_7b", "model_14b",
+__all__ = ["GIB", "LayerSpec", "Workload", "block_index", "tiny", "model_1p4b", "model_7b", "model_14b",
            "WORKLOADS", "DEQUANT_SHAPES", "workload", "layer_host", "layer_device",
            "normal_matrix_device", "random_bits_host", "bits_u16"]

@@ -425,3 +425,70 @@ def test_dq_score_nonfinite_tile_is_nan(cuda):
     assert math.isnan(oracle.layer_error_dq(bits(w), oracle.BF16)[2])
     assert math.isnan(rel.item())
     assert flag.item() == aqnf4.AQNF4_ERR_NONFINITE
+
+
+# ------------------------------------------------------------ block-level selection
+
+
+def _block_case(rng, L, B):
+    block_of = np.sort(rng.integers(0, B, L)).astype(np.int32)
+    sw = rng.uniform(0.5, 40.0, L)
+    se = rng.uniform(0.002, 0.05, L) * sw
+    cost = rng.integers(1, 1 << 30, L).astype(np.int64)
+    return se, sw, block_of, cost
+
+
+@pytest.mark.parametrize("order", [aqnf4.AQNF4_BLOCKS_BY_DEPTH, aqnf4.AQNF4_BLOCKS_BY_ERROR])
+@pytest.mark.parametrize("seed,L,B", [(0, 7, 3), (1, 224, 32), (2, 280, 40), (3, 3000, 1500),
+                                      (4, 5, 2048)])
+def test_select_blocks_matches_oracle(cuda, order, seed, L, B):
+    rng = np.random.default_rng(seed)
+    se, sw, block_of, cost = _block_case(rng, L, B)
+    if L > 10:
+        se[L // 3] = np.nan                          # a non-finite layer ranks its block last
+        se[L // 2] = se[L // 2 + 1] = 0.0            # equal scores
+        sw[L // 2] = sw[L // 2 + 1] = 1.0
+    total = int(cost.sum())
+    d = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(dt).to(cuda)
+    for budget in (0, total // 7, total // 2, total):
+        rank = torch.empty(B, dtype=torch.int32, device=cuda)
+        err = torch.empty(B, dtype=torch.float32, device=cuda)
+        k = torch.empty(1, dtype=torch.int32, device=cuda)
+        aqnf4.aqnf4_select_blocks(d(se, torch.float64), d(sw, torch.float64),
+                                  d(block_of, torch.int32), d(cost, torch.int64), B, budget,
+                                  order, rank, err, k)
+        orank, oerr, ok = oracle.select_blocks(se, sw, block_of, cost, B, budget, order)
+        assert same_float_bits(err.cpu().numpy(), oerr)
+        assert rank.cpu().tolist() == orank
+        assert k.item() == ok
+
+
+def test_select_blocks_on_scored_model(cuda):
+    """The 7B-shaped model's real scores, grouped by transformer block."""
+    wl = synth.workload("7b")
+    weights = [synth.layer_device(s, wl.seed, i, cuda) for i, s in enumerate(wl.layers)]
+    se, sw, _ = aqnf4.score_layers(weights)
+    del weights
+    block_of = torch.tensor(synth.block_index(wl), dtype=torch.int32, device=cuda)
+    cost = torch.tensor([aqnf4.aqnf4_cost_bytes(s.numel) for s in wl.layers], dtype=torch.int64,
+                        device=cuda)
+    B = int(block_of.max().item()) + 1
+    for order in (aqnf4.AQNF4_BLOCKS_BY_DEPTH, aqnf4.AQNF4_BLOCKS_BY_ERROR):
+        rank = torch.empty(B, dtype=torch.int32, device=cuda)
+        k = torch.empty(1, dtype=torch.int32, device=cuda)
+        aqnf4.aqnf4_select_blocks(se, sw, block_of, cost, B, wl.budgets[0], order, rank, None, k)
+        orank, _, ok = oracle.select_blocks(se.cpu().numpy(), sw.cpu().numpy(),
+                                            block_of.cpu().numpy(), cost.cpu().numpy(), B,
+                                            wl.budgets[0], order)
+        assert rank.cpu().tolist() == orank and k.item() == ok
+
+
+def test_select_blocks_reports_a_bad_block_index(cuda):
+    se = torch.ones(4, dtype=torch.float64, device=cuda)
+    block_of = torch.tensor([0, 1, 5, 1], dtype=torch.int32, device=cuda)
+    cost = torch.ones(4, dtype=torch.int64, device=cuda)
+    rank = torch.empty(2, dtype=torch.int32, device=cuda)
+    k = torch.empty(1, dtype=torch.int32, device=cuda)
+    aqnf4.aqnf4_select_blocks(se, se, block_of, cost, 2, 10, aqnf4.AQNF4_BLOCKS_BY_DEPTH, rank,
+                              None, k)
+    assert k.item() == -1
