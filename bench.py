@@ -370,6 +370,9 @@ def run_native(args):
     if world == 1:
         result["select_blocks"] = bench_select_blocks(wl, se, sw, cost, budget, dev, stream)
 
+    if world == 1:
+        result["split_model"] = bench_split_model(weights, budget, wl.k_cap, dev)
+
     if world == 1 and not args.no_dq_score:
         result["dq_score"] = bench_dq_score(weights, stor, wl, cost, budget, sel, k_sel, dev,
                                             stream, peak, steps=min(K, 100))
@@ -404,6 +407,22 @@ def run_native(args):
     if rank == 0:
         print(json.dumps(result), flush=True)
     return 0
+
+
+def bench_split_model(weights, budget, k_cap, dev):
+    """Materialize the split model once (fused pass + selection + keeping one copy per
+    layer): wall time including its allocations, and the memory report."""
+    import torch
+
+    from quantized_lora_setup_b200 import split_model
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    model = split_model.materialize(weights, budget, k_cap)
+    torch.cuda.synchronize(dev)
+    ms = (time.perf_counter() - t0) * 1e3
+    rep = model.memory_report()
+    del model
+    return {"wall_ms": ms, "memory": rep}
 
 
 def bench_select_blocks(wl, se, sw, cost, budget, dev, stream, reps=200):

@@ -1,0 +1,93 @@
+"""The split model (top-K layers in 16 bits, the rest NF4 + DQ) and its memory report.
+
+CPU: the byte accounting against the oracle's cost model.  GPU: materialize() against the
+oracle -- the kept set, every NF4 layer's dequantized weights bit for bit, the kept layers
+untouched, and the report's extra bytes equal to the kept layers' cost, within budget.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_lora_setup_b200 import aqnf4, split_model, synth
+
+DT = {torch.float16: oracle.F16, torch.bfloat16: oracle.BF16}
+
+
+def test_nf4_storage_bytes_closed_form():
+    for n in (1, 2, 63, 64, 65, 16383, 16384, 16385, 4096 * 11008, 5120 * 13824):
+        nb = -(-n // 64)
+        expect = -(-n // 2) + nb + 4 * -(-nb // 256)
+        assert split_model.nf4_storage_bytes(n) == expect
+        assert split_model.nf4_storage_bytes(n) == 2 * n - oracle.cost_bytes(n)
+        assert split_model.nf4_bytes(aqnf4.NF4Storage(n, "cpu")) == expect
+
+
+def test_memory_report_accounting_on_host_tensors():
+    """A hand-built split model: extra bytes = the kept layers' cost exactly."""
+    sizes = [(256, 256), (688, 256), (7, 13), (1, 1)]
+    layers = []
+    kept = [1, 2]
+    for i, shape in enumerate(sizes):
+        n = shape[0] * shape[1]
+        if i in kept:
+            w = torch.zeros(shape, dtype=torch.bfloat16)
+            layers.append(split_model.SplitLayer(i, "fp16", shape, w.dtype, 0.1, w, None))
+        else:
+            layers.append(split_model.SplitLayer(i, "nf4", shape, torch.bfloat16, 0.1, None,
+                                                 aqnf4.NF4Storage(n, "cpu")))
+    cost = sum(oracle.cost_bytes(sizes[i][0] * sizes[i][1]) for i in kept)
+    for budget, ok in ((cost, True), (cost - 1, False)):
+        rep = split_model.SplitModel(layers, [1, 2, 0, 3], kept, budget).memory_report()
+        assert rep["extra_bytes"] == cost
+        assert rep["total_bytes"] == rep["all_nf4_bytes"] + cost
+        assert rep["within_budget"] is ok
+        assert rep["fp16_layers"] == 2 and rep["layers"] == 4
+
+
+def _oracle_model(weights):
+    rel, dq = [], []
+    for w in weights:
+        b = synth.bits_u16(w.cpu())
+        rel.append(oracle.layer_error(b, DT[w.dtype])[2])
+        packed, absmax, _ = oracle.quantize(b, DT[w.dtype])
+        codes8, scales, _ = oracle.double_quant(absmax)
+        dq.append(oracle.dequantize(packed, b.size, DT[w.dtype], codes8=codes8, scales=scales))
+    return np.array(rel, np.float32), dq
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("budget_frac", [0.0, 0.3, 1.0])
+def test_materialize_tiny_model(cuda, budget_frac):
+    wl = synth.tiny(0)
+    weights = [synth.layer_host(s, wl.seed, i).to(cuda) for i, s in enumerate(wl.layers)]
+    cost = [aqnf4.aqnf4_cost_bytes(w.numel()) for w in weights]
+    budget = int(budget_frac * sum(cost))
+    model = split_model.materialize(weights, budget)
+    rel, dq = _oracle_model(weights)
+    assert model.kept == oracle.select_topk(rel, cost, budget)
+    for i, L in enumerate(model.layers):
+        w16 = model.weight(i)
+        assert tuple(w16.shape) == tuple(weights[i].shape)
+        if i in model.kept:
+            assert L.kind == "fp16" and w16.data_ptr() == weights[i].data_ptr()
+        else:
+            assert L.kind == "nf4"
+            got = synth.bits_u16(w16.cpu())
+            assert np.array_equal(got, dq[i]), i
+    rep = model.memory_report()
+    assert rep["extra_bytes"] == sum(cost[i] for i in model.kept)
+    assert rep["within_budget"] and rep["extra_bytes"] <= budget
+
+
+@pytest.mark.gpu
+def test_materialize_ranks_by_dq_score_when_asked(cuda):
+    wl = synth.tiny(1)
+    weights = [synth.layer_host(s, wl.seed, i).to(cuda) for i, s in enumerate(wl.layers)]
+    cost = [aqnf4.aqnf4_cost_bytes(w.numel()) for w in weights]
+    budget = sum(cost) // 4
+    model = split_model.materialize(weights, budget, dq_score=True)
+    rel = np.array([oracle.layer_error_dq(synth.bits_u16(w.cpu()), DT[w.dtype])[2]
+                    for w in weights], np.float32)
+    assert model.kept == oracle.select_topk(rel, cost, budget)
+    np.testing.assert_allclose([L.rel_err for L in model.layers], rel, rtol=1e-5)
