@@ -40,6 +40,9 @@ def load():
     lib.oracle_select_blocks.argtypes = [P, P, P, P, ctypes.c_int, ctypes.c_int, i64,
                                          ctypes.c_int, P, P, P]
     lib.oracle_select_blocks.restype = ctypes.c_int
+    lib.oracle_nf4_linear.argtypes = [P, ctypes.c_int, i64, i64, P, P, P, i64, ctypes.c_int,
+                                      P, P, P]
+    lib.oracle_nf4_linear.restype = ctypes.c_int
     lib.oracle_double_quant.argtypes = [P, i64, P, P, P]
     lib.oracle_double_quant.restype = None
     lib.oracle_dequantize.argtypes = [P, P, P, P, i64, ctypes.c_int, P, P]
@@ -166,6 +169,22 @@ def select_topk(rel_err, cost, budget: int, k_cap: int = -1):
     return [int(i) for i in sel[: k[0]]]
 
 
+def nf4_linear(x_bits, x_dtype, packed, codes8, scales, N: int, w_dtype, book=None):
+    """(y float64[M, N], yabs float64[M, N]) of y = x w_hat^T for x (M x K 16-bit bit patterns)
+    and the N x K layer stored as packed codes + codes8 + scales."""
+    levels, _ = book if book is not None else codebook()
+    x = np.ascontiguousarray(x_bits, np.uint16)
+    M, K = x.shape
+    y = np.zeros((M, N), np.float64)
+    yabs = np.zeros((M, N), np.float64)
+    if load().oracle_nf4_linear(_ptr(x), x_dtype, M, K, _ptr(np.ascontiguousarray(packed, np.uint8)),
+                                _ptr(np.ascontiguousarray(codes8, np.uint8)),
+                                _ptr(np.ascontiguousarray(scales, np.float32)), N, w_dtype,
+                                _ptr(levels), _ptr(y), _ptr(yabs)) != 0:
+        raise MemoryError("oracle_nf4_linear")
+    return y, yabs
+
+
 BLOCKS_BY_DEPTH = 0
 BLOCKS_BY_ERROR = 1
 
@@ -199,7 +218,7 @@ def dtype_bits_to_f32(bits, dtype):
 
 
 __all__ = ["F16", "BF16", "load", "default_pmax", "codebook", "quantize", "layer_error",
-           "layer_error_dq", "select_blocks", "BLOCKS_BY_DEPTH", "BLOCKS_BY_ERROR",
+           "layer_error_dq", "select_blocks", "nf4_linear", "BLOCKS_BY_DEPTH", "BLOCKS_BY_ERROR",
            "double_quant", "dequantize", "cost_bytes", "select_topk", "f32_to_dtype_bits",
            "dtype_bits_to_f32"]
 

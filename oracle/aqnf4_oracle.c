@@ -47,6 +47,7 @@
  *   - the DQ-absmax score (an option): the same error with w_hat reconstructed from the
  *     double-quantized constant a' = fl(fl(code8/255) * s) -- what a stored NF4 + DQ model
  *     dequantizes to -- while the codes still come from the binary32 absmax.
+ *   - linear layer on NF4 weights: y = x w_hat^T in binary64, w_hat rebuilt as dequantize does.
  *   - selection: sort by (score desc, index asc, NaN last); keep the longest prefix with
  *     at most k_cap layers and total incremental cost <= budget.
  */
@@ -403,6 +404,58 @@ void oracle_dequantize(const uint8_t* packed, const uint8_t* codes8, const float
     float prod = levels[code] * a;
     out[e] = or_round_to_dtype(prod, out_dtype);
   }
+}
+
+/* ------------------------------------------------ linear layer on NF4 weights */
+
+/* The forward product of a layer kept in NF4 + DQ ([QLoRA/HIW]: the 4-bit weights are
+   dequantized to 16 bits on the fly for the forward pass): y = x w_hat^T with
+   x: M x K 16-bit (x_dtype), row-major; w_hat: the N x K layer rebuilt in w_dtype from its
+   packed codes, codes8 and scales exactly as oracle_dequantize does; y: M x N in binary64
+   (every product and sum exact up to binary64 rounding).  yabs (optional) receives
+   sum_k |x_mk| |w_hat_nk|, the scale of the rounding error a binary32 accumulation may
+   make.  Returns 0, or -1 if memory runs out. */
+int oracle_nf4_linear(const uint16_t* x, int x_dtype, int64_t M, int64_t K,
+                      const uint8_t* packed, const uint8_t* codes8, const float* scales,
+                      int64_t N, int w_dtype, const float levels[16], double* y,
+                      double* yabs) {
+  uint16_t* row16 = (uint16_t*)calloc((size_t)K, sizeof(uint16_t));
+  double* wrow = (double*)calloc((size_t)K, sizeof(double));
+  double* xv = (double*)calloc((size_t)(M * K), sizeof(double));
+  if (!row16 || !wrow || !xv) {
+    free(row16);
+    free(wrow);
+    free(xv);
+    return -1;
+  }
+  for (int64_t i = 0; i < M * K; ++i) xv[i] = (double)or_load(x[i], x_dtype);
+  for (int64_t n = 0; n < N; ++n) {
+    /* row n of w_hat: elements n*K .. n*K + K - 1 of the flattened layer */
+    for (int64_t k = 0; k < K; ++k) {
+      int64_t e = n * K + k;
+      int64_t b = e / OR_BLOCK;
+      float frac = (float)codes8[b] / 255.0f;
+      float a = frac * scales[b / OR_DQ_BLOCK];
+      uint8_t byte = packed[e >> 1];
+      int code = (e & 1) == 0 ? (byte >> 4) : (byte & 15);
+      float prod = levels[code] * a;
+      row16[k] = or_round_to_dtype(prod, w_dtype);
+      wrow[k] = (double)or_load(row16[k], w_dtype);
+    }
+    for (int64_t m = 0; m < M; ++m) {
+      double acc = 0.0, aacc = 0.0;
+      for (int64_t k = 0; k < K; ++k) {
+        acc += xv[m * K + k] * wrow[k];
+        aacc += fabs(xv[m * K + k] * wrow[k]);
+      }
+      y[m * N + n] = acc;
+      if (yabs) yabs[m * N + n] = aacc;
+    }
+  }
+  free(row16);
+  free(wrow);
+  free(xv);
+  return 0;
 }
 
 /* ---------------------------------------------------------------- selection */

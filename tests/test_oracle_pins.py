@@ -477,6 +477,56 @@ def test_select_rules():
         oracle.select_topk(e, [1] * 5, -1)
 
 
+# ------------------------------------------------ linear layer on NF4 weights
+
+
+def _nf4_layer(rng, N, K, sigma=0.02, tdt=torch.bfloat16):
+    w = torch.from_numpy((rng.standard_normal((N, K)) * sigma).astype(np.float32)).to(tdt)
+    b = bits_of(w)
+    dt = oracle.BF16 if tdt == torch.bfloat16 else oracle.F16
+    packed, absmax, _ = oracle.quantize(b, dt)
+    codes8, scales, _ = oracle.double_quant(absmax)
+    return packed, codes8, scales
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 64), (5, 7, 128), (33, 20, 320)])
+def test_nf4_linear_equals_blas_on_dequantized_weights(M, N, K):
+    """y = x w_hat^T against numpy's BLAS product of the oracle's dequantized weights."""
+    rng = np.random.default_rng(M * 1000 + N)
+    packed, codes8, scales = _nf4_layer(rng, N, K)
+    x = torch.from_numpy(rng.standard_normal((M, K)).astype(np.float32)).to(torch.bfloat16)
+    y, yabs = oracle.nf4_linear(bits_of(x).reshape(M, K), oracle.BF16, packed, codes8, scales,
+                                N, oracle.BF16)
+    wq = oracle.dequantize(packed, N * K, oracle.BF16, codes8=codes8, scales=scales)
+    w64 = torch.from_numpy(wq.view(np.int16)).view(torch.bfloat16).double().numpy().reshape(N, K)
+    x64 = x.double().numpy()
+    ref = x64 @ w64.T
+    assert np.all(np.abs(y - ref) <= 1e-12 * np.maximum(yabs, 1e-300))
+    assert np.allclose(yabs, np.abs(x64) @ np.abs(w64).T, rtol=1e-12, atol=0)
+    assert np.all(yabs >= np.abs(y))
+
+
+def test_nf4_linear_exact_on_representable_weights():
+    """Weights NF4 + DQ store exactly -- bf16(level * 0.5), every block holding the maximum
+    0.5 so that code8 = 255 and a' = 0.5 -- and small integer activations: w_hat = w and the
+    product is exact in binary64."""
+    levels, _ = oracle.codebook()
+    rng = np.random.default_rng(3)
+    N, K, M = 6, 128, 4
+    codes = rng.integers(0, 16, (N, K))
+    codes[:, 0] = 15                                   # every block's maximum is 0.5
+    wb = torch.from_numpy((levels[codes] * np.float32(0.5)).astype(np.float32)).to(torch.bfloat16)
+    w = wb.float().numpy()
+    packed, absmax, _ = oracle.quantize(bits_of(wb), oracle.BF16)
+    codes8, scales, _ = oracle.double_quant(absmax)
+    assert np.all(codes8 == 255)
+    x = rng.integers(-3, 4, (M, K)).astype(np.float32)
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    y, _ = oracle.nf4_linear(bits_of(xb).reshape(M, K), oracle.BF16, packed, codes8, scales, N,
+                             oracle.BF16)
+    assert np.array_equal(y, x.astype(np.float64) @ w.astype(np.float64).T)
+
+
 # ------------------------------------------------------ block-level selection
 
 
