@@ -178,6 +178,24 @@ AQNF4_API aqnf4_status aqnf4_layer_error_noalloc(const aqnf4_layer* layers, int3
                                                  double* sq_err, double* sq_w, float* rel_err,
                                                  int32_t* dev_flag, cudaStream_t stream);
 
+/* Forward product of a layer stored in NF4 + DQ ("QLoRA", "How It Works": the 4-bit weights
+   are dequantized to 16 bits on the fly for the forward pass), on the tensor cores with the
+   dequantization fused in: y = x w_hat^T, where w_hat (N x K) is exactly what
+   aqnf4_dequantize(packed, codes8, scales, NULL, N*K, dtype, ...) returns for the layer's
+   storage, and the products are summed in binary32.
+   x (device, M x K, row-major, dtype, 16-byte aligned); packed (device, N*K/2 bytes,
+   16-byte aligned), codes8 (device, N*K/64 bytes), scales (device, ceil(N*K/16384) floats):
+   the layer's storage as aqnf4_layer_error writes it; y (device, M x N, row-major): float
+   when out_f32 != 0, else dtype.  K must be a positive multiple of 64, so that each row of
+   the layer is whole NF4 blocks.  dev_flag (optional, device int32) receives
+   AQNF4_ERR_TIMEOUT if a bounded wait inside the kernel gave up (y is then not written).
+   Errors: INVALID_ARG (NULL pointer, M < 1, N < 1, K not a positive multiple of 64, sizes
+   above 2^31), DTYPE, ALIGNMENT, CUDA. */
+AQNF4_API aqnf4_status aqnf4_nf4_linear(const void* x, int32_t dtype, int64_t M, int64_t K,
+                                        const uint8_t* packed, const uint8_t* codes8,
+                                        const float* scales, int64_t N, void* y,
+                                        int32_t out_f32, int32_t* dev_flag, cudaStream_t stream);
+
 /* Top-K under a byte budget (arxivdaily 2608.23816, "English abstract": keep the top-K in
    fp16 under a memory budget; "AQLoRA: ...", "Technical Details": configurable budget).
    Layers are ranked by rel_err descending, equal scores by lower index first, NaN scores

@@ -16,7 +16,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIB_DIR, "libaqnf4.so")
 SOURCES = ["codebook.cpp", "quant_score.cu", "double_quant.cu", "dequant.cu", "select.cu",
-           "selftest.cu"]
+           "selftest.cu", "nf4_gemm.cu"]
 HEADERS = ["internal.h", "device.cuh"]
 
 # -fmad=false: no multiply and add is ever fused behind the code's back (every FMA the

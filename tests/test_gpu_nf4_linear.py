@@ -1,0 +1,92 @@
+"""The fused NF4-dequant GEMM (aqnf4_nf4_linear) against the oracle's binary64 product.
+
+The layer's storage comes from the oracle (quantize + double quantization), so the kernel
+is checked independently of the library's own quantizer.  Bound: the kernel sums products
+that are exact in binary32 (16-bit times 16-bit), so any summation order stays within
+K * 2^-23 * sum |x w_hat| of the binary64 result; a 16-bit output adds its own rounding.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_lora_setup_b200 import aqnf4, synth
+
+
+DT = {torch.float16: oracle.F16, torch.bfloat16: oracle.BF16}
+
+
+def _case(M, N, K, dt, seed):
+    rng = np.random.default_rng(seed)
+    w = torch.from_numpy((rng.standard_normal((N, K)) * 0.02).astype(np.float32)).to(dt)
+    packed, absmax, _ = oracle.quantize(synth.bits_u16(w), DT[dt])
+    codes8, scales, _ = oracle.double_quant(absmax)
+    x = torch.from_numpy(rng.standard_normal((M, K)).astype(np.float32)).to(dt)
+    return x, packed, codes8, scales
+
+
+def _run(cuda, x, packed, codes8, scales, N, out_dtype):
+    M, K = x.shape
+    y = torch.full((M, N), float("nan"), dtype=out_dtype, device=cuda)
+    flag = torch.zeros(1, dtype=torch.int32, device=cuda)
+    aqnf4.aqnf4_nf4_linear(x.to(cuda), torch.from_numpy(packed).to(cuda),
+                           torch.from_numpy(codes8).to(cuda), torch.from_numpy(scales).to(cuda),
+                           N, y, flag)
+    torch.cuda.synchronize()
+    assert flag.item() == 0
+    return y.double().cpu().numpy()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("M,N,K", [(128, 128, 64), (1, 1, 64), (200, 300, 256),
+                                   (256, 384, 4096), (130, 129, 192)])
+def test_nf4_linear_matches_oracle(cuda, dt, M, N, K):
+    x, packed, codes8, scales = _case(M, N, K, dt, seed=M + N + K)
+    ref, rabs = oracle.nf4_linear(synth.bits_u16(x).reshape(M, K), DT[dt], packed, codes8,
+                                  scales, N, DT[dt])
+    bound = K * 2.0 ** -23 * rabs + 1e-30
+    y32 = _run(cuda, x, packed, codes8, scales, N, torch.float32)
+    assert np.all(np.abs(y32 - ref) <= bound)
+    y16 = _run(cuda, x, packed, codes8, scales, N, dt)
+    ulp = 2.0 ** -8 if dt == torch.bfloat16 else 2.0 ** -11
+    assert np.all(np.abs(y16 - ref) <= bound + ulp * (np.abs(ref) + bound) + 6e-8)
+
+
+@pytest.mark.gpu
+def test_nf4_linear_uses_the_library_storage(cuda):
+    """Storage written by the fused scoring pass (bit-equal to the oracle's) gives the same y."""
+    M, N, K = 64, 256, 512
+    rng = np.random.default_rng(9)
+    w = torch.from_numpy((rng.standard_normal((N, K)) * 0.02).astype(np.float32)).to(torch.bfloat16)
+    x, packed, codes8, scales = _case(M, N, K, torch.bfloat16, seed=9)
+    packed, absmax, _ = oracle.quantize(synth.bits_u16(w), oracle.BF16)
+    codes8, scales, _ = oracle.double_quant(absmax)
+    st = aqnf4.NF4Storage(N * K, cuda)
+    aqnf4.score_layers([w.reshape(-1).to(cuda)], [st])
+    torch.cuda.synchronize()
+    assert np.array_equal(st.packed.cpu().numpy(), packed)
+    assert np.array_equal(st.codes8.cpu().numpy(), codes8)
+    y_oracle_storage = _run(cuda, x, packed, codes8, scales, N, torch.float32)
+    y_lib_storage = _run(cuda, x, st.packed.cpu().numpy(), st.codes8.cpu().numpy(),
+                         st.scales.cpu().numpy(), N, torch.float32)
+    np.testing.assert_array_equal(y_lib_storage, y_oracle_storage)
+
+
+def test_nf4_linear_rejects_bad_shapes():
+    lib = aqnf4.library()
+    V = __import__("ctypes").c_void_p
+    before = lib.aqnf4_launch_count()
+    args = [V(0x1000), aqnf4.AQNF4_BF16, 4, 64, V(0x2000), V(0x3000), V(0x4000), 8, V(0x5000),
+            1, None, None]
+    for i, bad in ((3, 0), (3, 96), (3, 63), (2, 0), (7, 0), (0, None), (8, None)):
+        a = list(args)
+        a[i] = bad
+        assert lib.aqnf4_nf4_linear(*a) == aqnf4.AQNF4_ERR_INVALID_ARG, (i, bad)
+    a = list(args)
+    a[1] = 7
+    assert lib.aqnf4_nf4_linear(*a) == aqnf4.AQNF4_ERR_DTYPE
+    a = list(args)
+    a[0] = V(0x1008)
+    assert lib.aqnf4_nf4_linear(*a) == aqnf4.AQNF4_ERR_ALIGNMENT
+    assert lib.aqnf4_launch_count() == before
