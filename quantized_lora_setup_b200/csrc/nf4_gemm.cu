@@ -7,17 +7,23 @@
 //   a'_b = fl(fl(code8_b / 255) * scales[b / 256]),  w_hat = dtype_rn(fl(level[code] * a'_b)),
 // bit for bit what aqnf4_dequantize writes; then y = x w_hat^T with binary32 accumulation.
 //
-// Blackwell structure.  One CTA computes a 128 x 128 tile of y over K in steps of 64:
-//   - x (M x K, K contiguous) arrives by TMA in 128-byte-swizzled 128 x 64 tiles;
-//   - the 128 threads dequantize the matching 128 x 64 slice of w_hat -- thread t takes row
-//     n0 + t, which is exactly one NF4 block per step (K is a multiple of 64) -- and store it
-//     in the same swizzled K-major layout, 16 bytes at a time;
-//   - one thread issues four tcgen05.mma (M 128, N 128, K 16, bf16/f16 in, f32 out) per step
-//     into a TMEM accumulator, and tcgen05.commit frees the stage when they finish;
-//   - three stages let the dequantization and the x copy of the next steps overlap the
-//     tensor cores; the epilogue reads TMEM with tcgen05.ld (warp w owns lanes 32w..32w+31).
-// Every wait is bounded: a wait that gives up records AQNF4_ERR_TIMEOUT, lets the copies and
-// MMAs in flight finish (bounded too) and still frees the TMEM before the CTA exits.
+// Blackwell structure.  One CTA (18 warps, one per SM) computes a 256 x 256 tile of y over
+// K in steps of 64, its roles specialised and coupled only through mbarriers:
+//   - warp 16 streams, by TMA and up to three steps ahead, the step's x tile (M x K, K
+//     contiguous; 128-byte-swizzled 256 x 64) and the matching 256-row x 32-byte slice of the
+//     packed codes;
+//   - warps 0-15 dequantize that slice into a 256 x 64 w_hat tile -- threads 2r and 2r + 1
+//     take the two halves of row n0 + r, one NF4 block per row and step (K is a multiple of
+//     64) -- in the same swizzled K-major layout, 16 bytes at a time, and arrive on the
+//     stage's barrier; the 8-bit constants and DQ scales come two steps ahead from global;
+//   - warp 17 issues eight tcgen05.mma per step (M 128, N 256, K 16, bf16/f16 in, f32 out):
+//     each x row half against the same w_hat tile, into two TMEM accumulators that fill all
+//     512 columns, so every dequantized element feeds 256 rows of x; tcgen05.commit frees
+//     the stage when they finish;
+//   - warps 0-15 then read the accumulators with tcgen05.ld (warp w: TMEM lanes 32(w mod 4)..,
+//     accumulator w / 8, columns 128 ((w / 4) mod 2)..) and store y.
+// Every wait is bounded: a wait that gives up records AQNF4_ERR_TIMEOUT and makes every role
+// stop; copies in flight are allowed to land and the TMEM is always freed before exit.
 #include <cuda.h>
 
 #include <mutex>
@@ -27,13 +33,17 @@
 namespace aqnf4 {
 namespace {
 
-constexpr int kBM = 128, kBN = 128, kBK = 64, kStages = 3, kGThreads = 128;
-constexpr int kTileBytesA = kBM * kBK * 2;  // 16 KB
-constexpr int kTileBytesB = kBN * kBK * 2;  // 16 KB
-constexpr int kStageBytes = kTileBytesA + kTileBytesB;
-constexpr int kBarBase = kStages * kStageBytes;                // after the stages
-constexpr int kGSmemBytes = kBarBase + 256 + 1024;             // barriers + alignment slack
-constexpr uint32_t kTmemCols = 128;                            // f32 accumulator, 128 columns
+constexpr int kBM = 256, kBN = 256, kBK = 64, kStages = 3;  // two 128-row accumulators
+constexpr int kDeqWarps = 16, kProducerWarp = 16, kMmaWarp = 17;
+constexpr int kGThreads = 32 * (kDeqWarps + 2);            // 576
+constexpr int kTileBytesA = kBM * kBK * 2;                  // 32 KB of x
+constexpr int kTileBytesB = kBN * kBK * 2;                  // 32 KB of w_hat
+constexpr int kTileBytesP = kBN * kBK / 2;                  // 8 KB of packed codes
+constexpr int kStageBytes = kTileBytesA + kTileBytesB + kTileBytesP;
+constexpr int kBarBase = kStages * kStageBytes;             // after the stages
+constexpr int kGSmemBytes = kBarBase + 256 + 1024;          // barriers + alignment slack
+constexpr uint32_t kTmemCols = 512;  // two f32 accumulators of 256 columns: all of TMEM
+static_assert(kDeqWarps * 16 == kBN, "two dequantizing threads per row of the w_hat tile");
 
 struct GParams {
   const uint8_t* packed;
@@ -58,11 +68,11 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 }
 
 // Instruction descriptor: f32 accumulator, both operands DT (f16 = 0, bf16 = 1), K-major,
-// N = 128, M = 128.
+// N = 256, M = 128 (one of the two row halves of the tile).
 template <int DT>
 __host__ __device__ constexpr uint32_t idesc() {
   return (1u << 4) | (static_cast<uint32_t>(DT) << 7) | (static_cast<uint32_t>(DT) << 10) |
-         (static_cast<uint32_t>(kBN >> 3) << 17) | (static_cast<uint32_t>(kBM >> 4) << 24);
+         (static_cast<uint32_t>(kBN >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
@@ -81,6 +91,10 @@ __device__ __forceinline__ void umma_f16(uint32_t tmem, uint64_t da, uint64_t db
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
       "l"(da), "l"(db), "r"(id), "r"(accumulate)
       : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
@@ -116,34 +130,37 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 }
 
 template <int DT>
-__global__ void __launch_bounds__(kGThreads) k_nf4_gemm(const __grid_constant__ CUtensorMap tmap_x,
-                                                        const __grid_constant__ GParams p) {
+__global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant__ CUtensorMap tmap_x,
+                                                           const __grid_constant__ CUtensorMap tmap_w,
+                                                           const __grid_constant__ GParams p) {
   using F = Fmt<DT>;
   extern __shared__ uint8_t smem_raw[];
   // the swizzled tiles need 1024-byte alignment
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarBase);
-  uint64_t* empty = full + kStages;
+  uint64_t* full_a = reinterpret_cast<uint64_t*>(smem + kBarBase);
+  uint64_t* full_b = full_a + kStages;
+  uint64_t* empty = full_b + kStages;
   uint64_t* accum = empty + kStages;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accum + 1);
-  int* abort_flag = reinterpret_cast<int*>(tmem_holder + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kBN;
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kBM;
-  const float tab_level = p.level[lane & 15];  // lanes 16..31 mirror 0..15
+  const int64_t kb = p.K / kBK;  // NF4 blocks per row of w = k steps
 
   if (t == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_addr(full + s), 1);
+      mbar_init(smem_addr(full_a + s), 1);
+      mbar_init(smem_addr(full_b + s), 32 * kDeqWarps);
       mbar_init(smem_addr(empty + s), 1);
     }
     mbar_init(smem_addr(accum), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_addr(tmem_holder)),
                  "r"(kTmemCols)
@@ -155,89 +172,134 @@ __global__ void __launch_bounds__(kGThreads) k_nf4_gemm(const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  const int64_t kb = p.K / kBK;  // NF4 blocks per row of w = k steps
-  const int64_t n = n0 + t;      // this thread's row of w_hat
-  const bool row_ok = n < p.N;
-  int pend_stage = -1;           // thread 0: a copy whose completion it did not see
-  uint32_t pend_parity = 0;
+  int64_t last_kt[kStages];  // producer: the last step copied into each stage (-1: none)
+#pragma unroll
+  for (int s = 0; s < kStages; ++s) last_kt[s] = -1;
 
-  for (int64_t kt = 0; kt < kb; ++kt) {
-    const int s = static_cast<int>(kt % kStages);
-    const uint32_t use = static_cast<uint32_t>(kt / kStages);
-    uint8_t* sa = smem + s * kStageBytes;
-    uint8_t* sb = sa + kTileBytesA;
-    if (kt >= kStages && !mbar_wait_bounded(smem_addr(empty + s), (use - 1) & 1)) *abort_flag = 1;
-    __syncthreads();
-    if (*abort_flag) break;
-    if (t == 0) {
-      mbar_arrive_expect_tx(smem_addr(full + s), kTileBytesA);
-      tma_load_2d(smem_addr(sa), &tmap_x, static_cast<int>(kt * kBK), static_cast<int>(m0),
-                  smem_addr(full + s));
-    }
-    // ---- dequantize row n, k = kt*64 .. kt*64+63 (one NF4 block) into the swizzled tile
-    uint4 pk0 = make_uint4(0, 0, 0, 0), pk1 = pk0;
-    float ap = 0.0f;
-    if (row_ok) {
-      const int64_t b = n * kb + kt;
-      const uint4* src = reinterpret_cast<const uint4*>(p.packed + b * 32);
-      pk0 = __ldg(src);
-      pk1 = __ldg(src + 1);
-      ap = __fmul_rn(__fdiv_rn(static_cast<float>(__ldg(p.codes8 + b)), 255.0f),
-                     __ldg(p.scales + (b >> 8)));
-    }
-    const f32x2 a2 = pair(ap, ap);
-    const uint32_t words[8] = {pk0.x, pk0.y, pk0.z, pk0.w, pk1.x, pk1.y, pk1.z, pk1.w};
-    const int r = t;  // row within the tile
-    uint8_t* rowp = sb + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t w = words[j];
-      uint32_t o[4];
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        // byte h: element 2h in the high nibble, 2h + 1 in the low nibble
-        const float q0 = __shfl_sync(kFull, tab_level, static_cast<int>(w >> (8 * h + 4)));
-        const float q1 = __shfl_sync(kFull, tab_level, static_cast<int>(w >> (8 * h)));
-        const f32x2 v = pmul_rn(pair(q0, q1), a2);
-        o[h] = row_ok ? F::pack_rn(pair_lo(v), pair_hi(v)) : 0u;
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      for (int64_t kt = 0; kt < kb && !*abort_flag; ++kt) {
+        const int s = static_cast<int>(kt % kStages);
+        const uint32_t use = static_cast<uint32_t>(kt / kStages);
+        if (kt >= kStages && !mbar_wait_bounded(smem_addr(empty + s), (use - 1) & 1)) {
+          *abort_flag = 1;
+          break;
+        }
+        uint8_t* st = smem + s * kStageBytes;
+        mbar_arrive_expect_tx(smem_addr(full_a + s), kTileBytesA + kTileBytesP);
+        tma_load_2d(smem_addr(st), &tmap_x, static_cast<int>(kt * kBK), static_cast<int>(m0),
+                    smem_addr(full_a + s));
+        tma_load_2d(smem_addr(st + kTileBytesA + kTileBytesB), &tmap_w,
+                    static_cast<int>(kt * (kBK / 2)), static_cast<int>(n0), smem_addr(full_a + s));
+        last_kt[s] = kt;
       }
-      *reinterpret_cast<uint4*>(rowp + ((j ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
     }
-    fence_proxy_async_smem();  // the tensor cores read this tile through the async proxy
-    __syncthreads();
-    if (t == 0) {
-      if (!mbar_wait_bounded(smem_addr(full + s), use & 1)) {
-        *abort_flag = 1;
-        pend_stage = s;
-        pend_parity = use & 1;
-      } else {
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      for (int64_t kt = 0; kt < kb && !*abort_flag; ++kt) {
+        const int s = static_cast<int>(kt % kStages);
+        const uint32_t par = static_cast<uint32_t>(kt / kStages) & 1;
+        if (!mbar_wait_bounded(smem_addr(full_a + s), par) ||
+            !mbar_wait_bounded(smem_addr(full_b + s), par)) {
+          *abort_flag = 1;
+          break;
+        }
         tc_fence_after();
-        const uint32_t a0 = smem_addr(sa), b0 = smem_addr(sb);
+        const uint32_t a0 = smem_addr(smem + s * kStageBytes);
+        const uint32_t b0 = a0 + kTileBytesA;
 #pragma unroll
-        for (int j = 0; j < kBK / 16; ++j)  // K = 16 per MMA: 32 bytes along the swizzled row
+        for (int j = 0; j < kBK / 16; ++j) {  // K = 16 per MMA: 32 bytes along the swizzled row
+          // rows 0..127 of x into columns 0..255 of TMEM, rows 128..255 into 256..511; both
+          // use the same dequantized w_hat tile
           umma_f16(tmem, sw128_desc(a0 + 32 * j), sw128_desc(b0 + 32 * j), idesc<DT>(),
                    (kt > 0 || j > 0) ? 1u : 0u);
+          umma_f16(tmem + kBN, sw128_desc(a0 + 128 * 128 + 32 * j), sw128_desc(b0 + 32 * j),
+                   idesc<DT>(), (kt > 0 || j > 0) ? 1u : 0u);
+        }
         umma_commit(smem_addr(empty + s));
       }
+      umma_commit(smem_addr(accum));  // arrives once every MMA issued above has finished
+    }
+  } else {
+    // ---- dequantizing warps: threads 2r and 2r + 1 own the two halves of row n0 + r of the
+    // w_hat tile.  The packed codes arrive by TMA with x; the 8-bit constant and the DQ scale
+    // of steps kt + 1 and kt + 2 are loaded from global memory while step kt is worked on.
+    const float tab_level = p.level[lane & 15];  // lanes 16..31 mirror 0..15
+    const int r = t >> 1, hf = t & 1;
+    const int64_t n = n0 + r;
+    const bool row_ok = n < p.N;
+    // (code8, scale) of steps kt, kt + 1, kt + 2, rotated through registers
+    uint32_t c8_0 = 0, c8_1 = 0, c8_2 = 0;
+    float sc_0 = 0.0f, sc_1 = 0.0f, sc_2 = 0.0f;
+    auto fetch = [&](int64_t kt, uint32_t& c, float& s8) {
+      if (row_ok && kt < kb) {
+        const int64_t b = n * kb + kt;
+        c = __ldg(p.codes8 + b);
+        s8 = __ldg(p.scales + (b >> 8));
+      }
+    };
+    fetch(0, c8_0, sc_0);
+    fetch(1, c8_1, sc_1);
+    for (int64_t kt = 0; kt < kb; ++kt) {
+      const int s = static_cast<int>(kt % kStages);
+      const uint32_t use = static_cast<uint32_t>(kt / kStages);
+      c8_2 = 0;
+      sc_2 = 0.0f;
+      fetch(kt + 2, c8_2, sc_2);
+      bool ok = true;
+      if (kt >= kStages) ok = mbar_wait_bounded(smem_addr(empty + s), (use - 1) & 1);
+      ok = ok && mbar_wait_bounded(smem_addr(full_a + s), use & 1);  // packed codes landed
+      if (!ok) *abort_flag = 1;
+      if (__any_sync(kFull, *abort_flag != 0)) break;  // warp-uniform exit (shuffles below)
+      uint8_t* st = smem + s * kStageBytes;
+      const uint4 pk = *reinterpret_cast<const uint4*>(st + kTileBytesA + kTileBytesB + r * 32 + hf * 16);
+      // a zero constant (also for rows past N, whose codes are the copy's zero fill) gives 0
+      const float ap = row_ok ? __fmul_rn(__fdiv_rn(static_cast<float>(c8_0), 255.0f), sc_0)
+                              : 0.0f;
+      const f32x2 a2 = pair(ap, ap);
+      const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
+      uint8_t* rowb = st + kTileBytesA + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const uint32_t w = words[jj];
+        uint32_t o[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          // byte h: element 2h in the high nibble, 2h + 1 in the low nibble
+          const float q0 = __shfl_sync(kFull, tab_level, static_cast<int>(w >> (8 * h + 4)));
+          const float q1 = __shfl_sync(kFull, tab_level, static_cast<int>(w >> (8 * h)));
+          const f32x2 v = pmul_rn(pair(q0, q1), a2);
+          o[h] = F::pack_rn(pair_lo(v), pair_hi(v));
+        }
+        const int j = 4 * hf + jj;  // 16-byte chunk of the 128-byte row
+        *reinterpret_cast<uint4*>(rowb + ((j ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      fence_proxy_async_smem();  // the tensor cores read this tile through the async proxy
+      mbar_arrive(smem_addr(full_b + s));
+      c8_0 = c8_1;
+      sc_0 = sc_1;
+      c8_1 = c8_2;
+      sc_1 = sc_2;
     }
   }
 
-  // ---- all MMAs done -> accumulator ready (the decision is made uniformly: tcgen05.ld is a
-  // warp-collective instruction)
-  if (t == 0) umma_commit(smem_addr(accum));
-  const bool ready = mbar_wait_bounded(smem_addr(accum), 0);
+  // ---- accumulator ready?  (decided uniformly: tcgen05.ld is warp-collective)
+  const bool ready = warp < kDeqWarps ? mbar_wait_bounded(smem_addr(accum), 0) : true;
   const int failed = __syncthreads_or(!ready || *abort_flag);
   tc_fence_after();
   if (failed) {
     if (t == 0 && p.flag) *p.flag = AQNF4_ERR_TIMEOUT;
-  } else {
-    // ---- epilogue: warp w reads TMEM lanes 32w..32w+31 = rows m0 + 32w + lane
-    const int64_t m = m0 + 32 * warp + lane;
+  } else if (warp < kDeqWarps) {
+    // warp w: TMEM lanes 32 (w mod 4).. ; accumulator (w / 8) holds rows 128 (w / 8).. of the
+    // tile; columns 128 ((w / 4) mod 2)..
+    const int q = warp & 3, acc = warp >> 3, chalf = (warp >> 2) & 1;
+    const int64_t m = m0 + 128 * acc + 32 * q + lane;
 #pragma unroll 1
-    for (int c = 0; c < kBN / 32; ++c) {
+    for (int c = 0; c < 4; ++c) {
       float v[32];
-      tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 32 * c, v);
-      const int64_t col = n0 + 32 * c;
+      const int cbase = 128 * chalf + 32 * c;
+      tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + kBN * acc + cbase, v);
+      const int64_t col = n0 + cbase;
       if (m < p.M && col < p.N) {
         const bool whole = col + 32 <= p.N;
         if (p.out_f32) {
@@ -266,13 +328,15 @@ __global__ void __launch_bounds__(kGThreads) k_nf4_gemm(const __grid_constant__ 
       }
     }
   }
-  if (t == 0 && pend_stage >= 0) {
-    // let the copy that timed out land before the shared memory goes away
-    mbar_wait_bounded(smem_addr(full + pend_stage), pend_parity);
+  if (warp == kProducerWarp && lane == 0 && failed) {
+    // let every copy issued land before the shared memory goes away
+    for (int s = 0; s < kStages; ++s)
+      if (last_kt[s] >= 0)
+        mbar_wait_bounded(smem_addr(full_a + s), static_cast<uint32_t>(last_kt[s] / kStages) & 1);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(kTmemCols)
@@ -301,14 +365,15 @@ EncodeTiledFn encode_tiled() {
 }
 
 template <int DT>
-cudaError_t launch_gemm(const CUtensorMap& map, const GParams& p, cudaStream_t stream) {
+cudaError_t launch_gemm(const CUtensorMap& map, const CUtensorMap& wmap, const GParams& p,
+                        cudaStream_t stream) {
   auto kern = k_nf4_gemm<DT>;
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmemBytes);
   if (err != cudaSuccess) return err;
   const dim3 grid(static_cast<unsigned>((p.N + kBN - 1) / kBN),
                   static_cast<unsigned>((p.M + kBM - 1) / kBM));
-  kern<<<grid, kGThreads, kGSmemBytes, stream>>>(map, p);
+  kern<<<grid, kGThreads, kGSmemBytes, stream>>>(map, wmap, p);
   count_launches(1);
   return cudaGetLastError();
 }
@@ -346,6 +411,15 @@ extern "C" aqnf4_status aqnf4_nf4_linear(const void* x, int32_t dtype, int64_t M
              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return AQNF4_ERR_INVALID_ARG;
+  // packed codes as an N x K/2 byte matrix: a 256-row x 32-byte box is one step's slice
+  CUtensorMap wmap;
+  const cuuint64_t wdims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
+  const cuuint64_t wstrides[1] = {static_cast<cuuint64_t>(K / 2)};
+  const cuuint32_t wbox[2] = {kBK / 2, kBN};
+  if (encode(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), wdims,
+             wstrides, wbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return AQNF4_ERR_INVALID_ARG;
   GParams p;
   p.packed = packed;
   p.codes8 = codes8;
@@ -357,7 +431,7 @@ extern "C" aqnf4_status aqnf4_nf4_linear(const void* x, int32_t dtype, int64_t M
   p.out_f32 = out_f32 ? 1 : 0;
   p.flag = dev_flag;
   for (int i = 0; i < 16; ++i) p.level[i] = tb->level[i];
-  const cudaError_t err = dtype == AQNF4_BF16 ? launch_gemm<AQNF4_BF16>(map, p, stream)
-                                              : launch_gemm<AQNF4_F16>(map, p, stream);
+  const cudaError_t err = dtype == AQNF4_BF16 ? launch_gemm<AQNF4_BF16>(map, wmap, p, stream)
+                                              : launch_gemm<AQNF4_F16>(map, wmap, p, stream);
   return err == cudaSuccess ? AQNF4_OK : AQNF4_ERR_CUDA;
 }
