@@ -43,6 +43,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dequant", action="store_true")
+    ap.add_argument("--no-nf4-linear", action="store_true",
+                    help="skip the fused NF4-dequant GEMM measurement")
     ap.add_argument("--no-dq-score", action="store_true",
                     help="skip the step scored against the double-quantized constants")
     ap.add_argument("--extra-workloads", default="14b,1.4b",
@@ -373,6 +375,9 @@ def run_native(args):
     if world == 1:
         result["split_model"] = bench_split_model(weights, budget, wl.k_cap, dev)
 
+    if world == 1 and not args.no_nf4_linear:
+        result["nf4_linear"] = bench_nf4_linear(dev, stream)
+
     if world == 1 and not args.no_dq_score:
         result["dq_score"] = bench_dq_score(weights, stor, wl, cost, budget, sel, k_sel, dev,
                                             stream, peak, steps=min(K, 100))
@@ -407,6 +412,65 @@ def run_native(args):
     if rank == 0:
         print(json.dumps(result), flush=True)
     return 0
+
+
+def measured_tensor_peak():
+    """(dense bf16 TFLOP/s for a kernel timed in a short burst, source)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback"
+
+
+def bench_nf4_linear(dev, stream, reps=20):
+    """The forward product of an NF4 + DQ layer, y = x w_hat^T, with the dequantization fused
+    into the tcgen05 GEMM (aqnf4_nf4_linear): the 7B-shaped MLP up-projection (11008 x 4096)
+    at 4096 and 128 tokens, bf16.  TFLOP/s against the measured bf16 peak, beside the unfused
+    path (aqnf4_dequantize, then cuBLAS on the bf16 weights) for context."""
+    import torch
+
+    from quantized_lora_setup_b200 import aqnf4, synth
+    peak, src = measured_tensor_peak()
+    N, K = 11008, 4096
+    w = synth.normal_matrix_device(N, K, seed=7, device=dev)
+    st = aqnf4.NF4Storage(N * K, dev)
+    aqnf4.score_layers([w.reshape(-1)], [st], stream=stream)
+    del w
+    wd = torch.empty(N * K, dtype=torch.bfloat16, device=dev)
+    out = {"layer": [N, K], "unit": "TFLOP/s", "peak": peak, "peak_source": f"{src} bf16_tflops"}
+    for M in (4096, 128):
+        g = torch.Generator(device=dev)
+        g.manual_seed(M)
+        x = torch.randn((M, K), generator=g, device=dev).to(torch.bfloat16)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+
+        def fused():
+            aqnf4.aqnf4_nf4_linear(x, st.packed, st.codes8, st.scales, N, y, None, stream)
+
+        def unfused():
+            aqnf4.aqnf4_dequantize(st.packed, st.codes8, st.scales, None, N * K, wd, stream)
+            torch.matmul(x, wd.view(N, K).t(), out=y)
+
+        res = {}
+        for name, fn in (("fused", fused), ("dequant_then_cublas", unfused)):
+            for _ in range(3):
+                fn()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            ms = a.elapsed_time(b) / reps
+            res[name] = 2.0 * M * N * K / (ms / 1e3) / 1e12
+        out[f"tokens_{M}"] = {
+            "value": res["fused"], "ms": 2.0 * M * N * K / res["fused"] / 1e9,
+            "roofline": {"bound": "tensor", "achieved": res["fused"], "peak": peak,
+                         "unit": "TFLOP/s", "frac": res["fused"] / peak,
+                         "kernel": "k_nf4_gemm"},
+            "dequant_then_cublas": res["dequant_then_cublas"]}
+    return out
 
 
 def bench_split_model(weights, budget, k_cap, dev):

@@ -41,7 +41,8 @@ constexpr int kTileBytesB = kBN * kBK * 2;                  // 32 KB of w_hat
 constexpr int kTileBytesP = kBN * kBK / 2;                  // 8 KB of packed codes
 constexpr int kStageBytes = kTileBytesA + kTileBytesB + kTileBytesP;
 constexpr int kBarBase = kStages * kStageBytes;             // after the stages
-constexpr int kGSmemBytes = kBarBase + 256 + 1024;          // barriers + alignment slack
+constexpr int kFracOff = kBarBase + 256;                     // fl(c / 255) for c = 0..255
+constexpr int kGSmemBytes = kFracOff + 1024 + 1024;         // + alignment slack
 constexpr uint32_t kTmemCols = 512;  // two f32 accumulators of 256 columns: all of TMEM
 static_assert(kDeqWarps * 16 == kBN, "two dequantizing threads per row of the w_hat tile");
 
@@ -144,6 +145,8 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
   uint64_t* accum = empty + kStages;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accum + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  float* frac = reinterpret_cast<float*>(smem + kFracOff);
+  if (t < 256) frac[t] = __fdiv_rn(static_cast<float>(t), 255.0f);  // correctly rounded
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kBN;
@@ -254,8 +257,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
       uint8_t* st = smem + s * kStageBytes;
       const uint4 pk = *reinterpret_cast<const uint4*>(st + kTileBytesA + kTileBytesB + r * 32 + hf * 16);
       // a zero constant (also for rows past N, whose codes are the copy's zero fill) gives 0
-      const float ap = row_ok ? __fmul_rn(__fdiv_rn(static_cast<float>(c8_0), 255.0f), sc_0)
-                              : 0.0f;
+      const float ap = row_ok ? __fmul_rn(frac[c8_0], sc_0) : 0.0f;
       const f32x2 a2 = pair(ap, ap);
       const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
       uint8_t* rowb = st + kTileBytesA + (r >> 3) * 1024 + (r & 7) * 128;
