@@ -146,9 +146,9 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accum + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   float* frac = reinterpret_cast<float*>(smem + kFracOff);
-  if (t < 256) frac[t] = __fdiv_rn(static_cast<float>(t), 255.0f);  // correctly rounded
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  if (t < 256) frac[t] = __fdiv_rn(static_cast<float>(t), 255.0f);  // correctly rounded
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kBN;
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kBM;
   const int64_t kb = p.K / kBK;  // NF4 blocks per row of w = k steps
