@@ -45,6 +45,11 @@ def parse_args():
     ap.add_argument("--no-dequant", action="store_true")
     ap.add_argument("--no-nf4-linear", action="store_true",
                     help="skip the fused NF4-dequant GEMM measurement")
+    ap.add_argument("--only-nf4-linear", action="store_true",
+                    help="time only the fused NF4-dequant GEMM (shape: --gemm-shape)")
+    ap.add_argument("--gemm-shape", default="4096,11008,4096",
+                    help="M,N,K of --only-nf4-linear")
+    ap.add_argument("--gemm-reps", type=int, default=20)
     ap.add_argument("--no-dq-score", action="store_true",
                     help="skip the step scored against the double-quantized constants")
     ap.add_argument("--extra-workloads", default="14b,1.4b",
@@ -423,7 +428,20 @@ def measured_tensor_peak():
         return 1590.0, "fallback"
 
 
-def bench_nf4_linear(dev, stream, reps=20):
+def run_only_nf4_linear(args):
+    """One JSON line with the fused GEMM alone (for profiling a single shape)."""
+    import torch
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    M, N, K = (int(v) for v in args.gemm_shape.split(","))
+    out = bench_nf4_linear(dev, torch.cuda.current_stream(dev), reps=args.gemm_reps,
+                           shapes=((M, N, K),), baseline=False)
+    print(json.dumps({"nf4_linear": out}), flush=True)
+    return 0
+
+
+def bench_nf4_linear(dev, stream, reps=20, shapes=((4096, 11008, 4096), (128, 11008, 4096)),
+                     baseline=True):
     """The forward product of an NF4 + DQ layer, y = x w_hat^T, with the dequantization fused
     into the tcgen05 GEMM (aqnf4_nf4_linear): the 7B-shaped MLP up-projection (11008 x 4096)
     at 4096 and 128 tokens, bf16.  TFLOP/s against the measured bf16 peak, beside the unfused
@@ -432,28 +450,35 @@ def bench_nf4_linear(dev, stream, reps=20):
 
     from quantized_lora_setup_b200 import aqnf4, synth
     peak, src = measured_tensor_peak()
-    N, K = 11008, 4096
-    w = synth.normal_matrix_device(N, K, seed=7, device=dev)
-    st = aqnf4.NF4Storage(N * K, dev)
-    aqnf4.score_layers([w.reshape(-1)], [st], stream=stream)
-    del w
-    wd = torch.empty(N * K, dtype=torch.bfloat16, device=dev)
-    out = {"layer": [N, K], "unit": "TFLOP/s", "peak": peak, "peak_source": f"{src} bf16_tflops"}
-    for M in (4096, 128):
+    out = {"unit": "TFLOP/s", "peak": peak, "peak_source": f"{src} bf16_tflops"}
+    layers = {}
+    for M, N, K in shapes:
+        if (N, K) not in layers:
+            w = synth.normal_matrix_device(N, K, seed=7, device=dev)
+            st = aqnf4.NF4Storage(N * K, dev)
+            aqnf4.score_layers([w.reshape(-1)], [st], stream=stream)
+            del w
+            layers[(N, K)] = st
+        st = layers[(N, K)]
+        out["layer"] = [N, K]
+        wd = torch.empty(N * K, dtype=torch.bfloat16, device=dev) if baseline else None
         g = torch.Generator(device=dev)
         g.manual_seed(M)
         x = torch.randn((M, K), generator=g, device=dev).to(torch.bfloat16)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(max(16, aqnf4.aqnf4_nf4_linear_workspace_size(M, N, K)),
+                         dtype=torch.uint8, device=dev)
 
         def fused():
-            aqnf4.aqnf4_nf4_linear(x, st.packed, st.codes8, st.scales, N, y, None, stream)
+            aqnf4.aqnf4_nf4_linear(x, st.packed, st.codes8, st.scales, N, y, None, stream, ws)
 
         def unfused():
             aqnf4.aqnf4_dequantize(st.packed, st.codes8, st.scales, None, N * K, wd, stream)
             torch.matmul(x, wd.view(N, K).t(), out=y)
 
         res = {}
-        for name, fn in (("fused", fused), ("dequant_then_cublas", unfused)):
+        arms = (("fused", fused), ("dequant_then_cublas", unfused)) if baseline else (("fused", fused),)
+        for name, fn in arms:
             for _ in range(3):
                 fn()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -466,10 +491,11 @@ def bench_nf4_linear(dev, stream, reps=20):
             res[name] = 2.0 * M * N * K / (ms / 1e3) / 1e12
         out[f"tokens_{M}"] = {
             "value": res["fused"], "ms": 2.0 * M * N * K / res["fused"] / 1e9,
+            "split_k": aqnf4.aqnf4_nf4_linear_workspace_size(M, N, K) > 0,
             "roofline": {"bound": "tensor", "achieved": res["fused"], "peak": peak,
                          "unit": "TFLOP/s", "frac": res["fused"] / peak,
                          "kernel": "k_nf4_gemm"},
-            "dequant_then_cublas": res["dequant_then_cublas"]}
+            "dequant_then_cublas": res.get("dequant_then_cublas")}
     return out
 
 
@@ -705,6 +731,8 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.only_nf4_linear:
+        return run_only_nf4_linear(args)
     return run_native(args)
 
 

@@ -94,8 +94,11 @@ def library() -> ctypes.CDLL:
     lib.aqnf4_select_topk.restype = st
     lib.aqnf4_selftest_wait_timeout.argtypes = [i64, P, P, P]
     lib.aqnf4_selftest_wait_timeout.restype = st
-    lib.aqnf4_nf4_linear.argtypes = [P, i32, i64, i64, P, P, P, i64, P, i32, P, P]
+    lib.aqnf4_nf4_linear.argtypes = [P, i32, i64, i64, P, P, P, i64, P, i32, P,
+                                     ctypes.c_size_t, P, P]
     lib.aqnf4_nf4_linear.restype = st
+    lib.aqnf4_nf4_linear_workspace_size.argtypes = [i64, i64, i64]
+    lib.aqnf4_nf4_linear_workspace_size.restype = ctypes.c_size_t
     lib.aqnf4_select_blocks.argtypes = [P, P, P, P, i32, i32, i64, i32, P, P, P, P]
     lib.aqnf4_select_blocks.restype = st
     lib.aqnf4_slot_tables.argtypes = [P, P, P]
@@ -229,16 +232,23 @@ def aqnf4_selftest_wait_timeout(timeout_ns: int, dev_flag: torch.Tensor,
 
 def aqnf4_nf4_linear(x: torch.Tensor, packed: torch.Tensor, codes8: torch.Tensor,
                      scales: torch.Tensor, N: int, y: torch.Tensor,
-                     dev_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+                     dev_flag: Optional[torch.Tensor] = None, stream=None,
+                     workspace: Optional[torch.Tensor] = None) -> None:
     """y (M x N) = x (M x K) w_hat^T for the N x K layer stored as packed + codes8 + scales;
-    y may be float32 or x's dtype."""
+    y may be float32 or x's dtype.  workspace: see aqnf4_nf4_linear_workspace_size."""
     M, K = x.shape
     out_f32 = 1 if y.dtype == torch.float32 else 0
     if not out_f32 and y.dtype != x.dtype:
         raise ValueError("y must be float32 or x's dtype")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(library().aqnf4_nf4_linear(_ptr(x), dtype_code(x.dtype), M, K, _ptr(packed),
                                       _ptr(codes8), _ptr(scales), N, _ptr(y), out_f32,
-                                      _ptr(dev_flag), _stream(stream)), "aqnf4_nf4_linear")
+                                      _ptr(workspace), ws_bytes, _ptr(dev_flag),
+                                      _stream(stream)), "aqnf4_nf4_linear")
+
+
+def aqnf4_nf4_linear_workspace_size(M: int, N: int, K: int) -> int:
+    return int(library().aqnf4_nf4_linear_workspace_size(M, N, K))
 
 
 def aqnf4_select_blocks(sq_err: torch.Tensor, sq_w: torch.Tensor, block_of: torch.Tensor,

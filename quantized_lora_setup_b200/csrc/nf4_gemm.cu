@@ -53,6 +53,8 @@ struct GParams {
   void* y;
   int64_t M, N, K;
   int32_t out_f32;
+  int32_t splits;  // K is split over gridDim.z CTAs; > 1: partial sums go to ws
+  float* ws;       // [splits][M][N] binary32 partial sums (splits > 1)
   int32_t* flag;
   float level[16];
 };
@@ -152,6 +154,10 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kBN;
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kBM;
   const int64_t kb = p.K / kBK;  // NF4 blocks per row of w = k steps
+  // this CTA's steps [kt0, kt1): split z of p.splits (the pipeline counts i = kt - kt0)
+  const int64_t kt0 = kb * blockIdx.z / p.splits, kt1 = kb * (blockIdx.z + 1) / p.splits;
+  const int64_t nk = kt1 - kt0;
+  const bool lower_half = m0 + 128 < p.M;  // the tile's second 128 rows hold any of x
 
   if (t == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -181,10 +187,11 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
-      for (int64_t kt = 0; kt < kb && !*abort_flag; ++kt) {
-        const int s = static_cast<int>(kt % kStages);
-        const uint32_t use = static_cast<uint32_t>(kt / kStages);
-        if (kt >= kStages && !mbar_wait_bounded(smem_addr(empty + s), (use - 1) & 1)) {
+      for (int64_t i = 0; i < nk && !*abort_flag; ++i) {
+        const int64_t kt = kt0 + i;
+        const int s = static_cast<int>(i % kStages);
+        const uint32_t use = static_cast<uint32_t>(i / kStages);
+        if (i >= kStages && !mbar_wait_bounded(smem_addr(empty + s), (use - 1) & 1)) {
           *abort_flag = 1;
           break;
         }
@@ -194,14 +201,14 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
                     smem_addr(full_a + s));
         tma_load_2d(smem_addr(st + kTileBytesA + kTileBytesB), &tmap_w,
                     static_cast<int>(kt * (kBK / 2)), static_cast<int>(n0), smem_addr(full_a + s));
-        last_kt[s] = kt;
+        last_kt[s] = i;
       }
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
-      for (int64_t kt = 0; kt < kb && !*abort_flag; ++kt) {
-        const int s = static_cast<int>(kt % kStages);
-        const uint32_t par = static_cast<uint32_t>(kt / kStages) & 1;
+      for (int64_t i = 0; i < nk && !*abort_flag; ++i) {
+        const int s = static_cast<int>(i % kStages);
+        const uint32_t par = static_cast<uint32_t>(i / kStages) & 1;
         if (!mbar_wait_bounded(smem_addr(full_a + s), par) ||
             !mbar_wait_bounded(smem_addr(full_b + s), par)) {
           *abort_flag = 1;
@@ -215,9 +222,10 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
           // rows 0..127 of x into columns 0..255 of TMEM, rows 128..255 into 256..511; both
           // use the same dequantized w_hat tile
           umma_f16(tmem, sw128_desc(a0 + 32 * j), sw128_desc(b0 + 32 * j), idesc<DT>(),
-                   (kt > 0 || j > 0) ? 1u : 0u);
-          umma_f16(tmem + kBN, sw128_desc(a0 + 128 * 128 + 32 * j), sw128_desc(b0 + 32 * j),
-                   idesc<DT>(), (kt > 0 || j > 0) ? 1u : 0u);
+                   (i > 0 || j > 0) ? 1u : 0u);
+          if (lower_half)  // uniform: skipped when those 128 rows lie past M
+            umma_f16(tmem + kBN, sw128_desc(a0 + 128 * 128 + 32 * j), sw128_desc(b0 + 32 * j),
+                     idesc<DT>(), (i > 0 || j > 0) ? 1u : 0u);
         }
         umma_commit(smem_addr(empty + s));
       }
@@ -235,22 +243,23 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
     uint32_t c8_0 = 0, c8_1 = 0, c8_2 = 0;
     float sc_0 = 0.0f, sc_1 = 0.0f, sc_2 = 0.0f;
     auto fetch = [&](int64_t kt, uint32_t& c, float& s8) {
-      if (row_ok && kt < kb) {
+      if (row_ok && kt < kt1) {
         const int64_t b = n * kb + kt;
         c = __ldg(p.codes8 + b);
         s8 = __ldg(p.scales + (b >> 8));
       }
     };
-    fetch(0, c8_0, sc_0);
-    fetch(1, c8_1, sc_1);
-    for (int64_t kt = 0; kt < kb; ++kt) {
-      const int s = static_cast<int>(kt % kStages);
-      const uint32_t use = static_cast<uint32_t>(kt / kStages);
+    fetch(kt0, c8_0, sc_0);
+    fetch(kt0 + 1, c8_1, sc_1);
+    for (int64_t i = 0; i < nk; ++i) {
+      const int64_t kt = kt0 + i;
+      const int s = static_cast<int>(i % kStages);
+      const uint32_t use = static_cast<uint32_t>(i / kStages);
       c8_2 = 0;
       sc_2 = 0.0f;
       fetch(kt + 2, c8_2, sc_2);
       bool ok = true;
-      if (kt >= kStages) ok = mbar_wait_bounded(smem_addr(empty + s), (use - 1) & 1);
+      if (i >= kStages) ok = mbar_wait_bounded(smem_addr(empty + s), (use - 1) & 1);
       ok = ok && mbar_wait_bounded(smem_addr(full_a + s), use & 1);  // packed codes landed
       if (!ok) *abort_flag = 1;
       if (__any_sync(kFull, *abort_flag != 0)) break;  // warp-uniform exit (shuffles below)
@@ -304,8 +313,9 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
       const int64_t col = n0 + cbase;
       if (m < p.M && col < p.N) {
         const bool whole = col + 32 <= p.N;
-        if (p.out_f32) {
-          float* dst = static_cast<float*>(p.y) + m * p.N + col;
+        if (p.splits > 1 || p.out_f32) {
+          float* dst = p.splits > 1 ? p.ws + (blockIdx.z * p.M + m) * p.N + col
+                                    : static_cast<float*>(p.y) + m * p.N + col;
           if (whole && (p.N & 3) == 0) {
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
@@ -346,6 +356,35 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
   }
 }
 
+// Split K: y = sum over z of the binary32 partials ws[z], added in split order (the result
+// does not depend on scheduling), converted to y's format.
+template <int DT>
+__global__ void __launch_bounds__(256) k_splitk_reduce(const float* __restrict__ ws, int splits,
+                                                       int64_t mn, void* y, int out_f32) {
+  using F = Fmt<DT>;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < mn;
+       i += static_cast<int64_t>(gridDim.x) * 256) {
+    float acc = __ldcs(ws + i);
+    for (int z = 1; z < splits; ++z) acc = __fadd_rn(acc, __ldcs(ws + z * mn + i));
+    if (out_f32)
+      static_cast<float*>(y)[i] = acc;
+    else
+      static_cast<uint16_t*>(y)[i] = static_cast<uint16_t>(F::pack_rn(acc, 0.0f) & 0xffffu);
+  }
+}
+
+// Splits of K for a grid too small to fill the GPU: enough CTAs for one wave, at least 8
+// steps of 64 per split, at most 16 splits.
+int choose_splits(int64_t M, int64_t N, int64_t K) {
+  const int sms = current_sm_count() > 0 ? current_sm_count() : 148;
+  const int64_t tiles = ((N + kBN - 1) / kBN) * ((M + kBM - 1) / kBM);
+  if (tiles >= sms) return 1;
+  int64_t s = sms / tiles;
+  s = s < (K / kBK) / 8 ? s : (K / kBK) / 8;
+  s = s < 16 ? s : 16;
+  return s >= 2 ? static_cast<int>(s) : 1;
+}
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -374,9 +413,18 @@ cudaError_t launch_gemm(const CUtensorMap& map, const CUtensorMap& wmap, const G
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmemBytes);
   if (err != cudaSuccess) return err;
   const dim3 grid(static_cast<unsigned>((p.N + kBN - 1) / kBN),
-                  static_cast<unsigned>((p.M + kBM - 1) / kBM));
+                  static_cast<unsigned>((p.M + kBM - 1) / kBM), static_cast<unsigned>(p.splits));
   kern<<<grid, kGThreads, kGSmemBytes, stream>>>(map, wmap, p);
   count_launches(1);
+  if (p.splits > 1) {
+    const int64_t mn = p.M * p.N;
+    int64_t blocks = (mn + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(current_sm_count() > 0 ? current_sm_count() : 148) * 8;
+    if (blocks > cap) blocks = cap;
+    k_splitk_reduce<DT><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p.ws, p.splits, mn,
+                                                                           p.y, p.out_f32);
+    count_launches(1);
+  }
   return cudaGetLastError();
 }
 
@@ -385,11 +433,17 @@ cudaError_t launch_gemm(const CUtensorMap& map, const CUtensorMap& wmap, const G
 
 using namespace aqnf4;
 
+extern "C" size_t aqnf4_nf4_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || N < 1 || K < kBK || K % kBK != 0) return 0;
+  const int s = choose_splits(M, N, K);
+  return s > 1 ? static_cast<size_t>(s) * static_cast<size_t>(M) * static_cast<size_t>(N) * 4 : 0;
+}
+
 extern "C" aqnf4_status aqnf4_nf4_linear(const void* x, int32_t dtype, int64_t M, int64_t K,
                                          const uint8_t* packed, const uint8_t* codes8,
                                          const float* scales, int64_t N, void* y,
-                                         int32_t out_f32, int32_t* dev_flag,
-                                         cudaStream_t stream) {
+                                         int32_t out_f32, void* workspace, size_t ws_bytes,
+                                         int32_t* dev_flag, cudaStream_t stream) {
   if (!x || !packed || !codes8 || !scales || !y || M < 1 || N < 1 || K < kBK || K % kBK != 0)
     return AQNF4_ERR_INVALID_ARG;
   if (M > (int64_t(1) << 31) - kBM || N > (int64_t(1) << 31) - kBN || K > (int64_t(1) << 31))
@@ -431,6 +485,11 @@ extern "C" aqnf4_status aqnf4_nf4_linear(const void* x, int32_t dtype, int64_t M
   p.N = N;
   p.K = K;
   p.out_f32 = out_f32 ? 1 : 0;
+  p.splits = choose_splits(M, N, K);
+  p.ws = static_cast<float*>(workspace);
+  if (p.splits > 1 && (!workspace || !is_aligned(workspace, 16) ||
+                       ws_bytes < static_cast<size_t>(p.splits) * M * N * 4))
+    p.splits = 1;  // no room for the partial sums: one CTA per output tile
   p.flag = dev_flag;
   for (int i = 0; i < 16; ++i) p.level[i] = tb->level[i];
   const cudaError_t err = dtype == AQNF4_BF16 ? launch_gemm<AQNF4_BF16>(map, wmap, p, stream)

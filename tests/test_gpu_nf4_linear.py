@@ -25,13 +25,17 @@ def _case(M, N, K, dt, seed):
     return x, packed, codes8, scales
 
 
-def _run(cuda, x, packed, codes8, scales, N, out_dtype):
+def _run(cuda, x, packed, codes8, scales, N, out_dtype, split=True):
     M, K = x.shape
     y = torch.full((M, N), float("nan"), dtype=out_dtype, device=cuda)
     flag = torch.zeros(1, dtype=torch.int32, device=cuda)
+    ws = None
+    if split:
+        nbytes = aqnf4.aqnf4_nf4_linear_workspace_size(M, N, K)
+        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=cuda)
     aqnf4.aqnf4_nf4_linear(x.to(cuda), torch.from_numpy(packed).to(cuda),
                            torch.from_numpy(codes8).to(cuda), torch.from_numpy(scales).to(cuda),
-                           N, y, flag)
+                           N, y, flag, workspace=ws)
     torch.cuda.synchronize()
     assert flag.item() == 0
     return y.double().cpu().numpy()
@@ -51,6 +55,24 @@ def test_nf4_linear_matches_oracle(cuda, dt, M, N, K):
     y16 = _run(cuda, x, packed, codes8, scales, N, dt)
     ulp = 2.0 ** -8 if dt == torch.bfloat16 else 2.0 ** -11
     assert np.all(np.abs(y16 - ref) <= bound + ulp * (np.abs(ref) + bound) + 6e-8)
+    # without a workspace the call runs unsplit: same bound
+    y32u = _run(cuda, x, packed, codes8, scales, N, torch.float32, split=False)
+    assert np.all(np.abs(y32u - ref) <= bound)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("M,N,K", [(128, 11008, 4096), (16, 1024, 2048), (300, 512, 8192)])
+def test_nf4_linear_split_k_matches_oracle(cuda, M, N, K):
+    """Few output tiles: K is split over several CTAs whose partials are added in order."""
+    assert aqnf4.aqnf4_nf4_linear_workspace_size(M, N, K) > 0
+    x, packed, codes8, scales = _case(M, N, K, torch.bfloat16, seed=K + M)
+    ref, rabs = oracle.nf4_linear(synth.bits_u16(x).reshape(M, K), oracle.BF16, packed, codes8,
+                                  scales, N, oracle.BF16)
+    bound = K * 2.0 ** -23 * rabs + 1e-30
+    y1 = _run(cuda, x, packed, codes8, scales, N, torch.float32)
+    y2 = _run(cuda, x, packed, codes8, scales, N, torch.float32)
+    assert np.all(np.abs(y1 - ref) <= bound)
+    assert np.array_equal(y1, y2)  # the partial sums are added in a fixed order
 
 
 @pytest.mark.gpu
@@ -78,7 +100,7 @@ def test_nf4_linear_rejects_bad_shapes():
     V = __import__("ctypes").c_void_p
     before = lib.aqnf4_launch_count()
     args = [V(0x1000), aqnf4.AQNF4_BF16, 4, 64, V(0x2000), V(0x3000), V(0x4000), 8, V(0x5000),
-            1, None, None]
+            1, None, 0, None, None]
     for i, bad in ((3, 0), (3, 96), (3, 63), (2, 0), (7, 0), (0, None), (8, None)):
         a = list(args)
         a[i] = bad
@@ -90,3 +112,4 @@ def test_nf4_linear_rejects_bad_shapes():
     a[0] = V(0x1008)
     assert lib.aqnf4_nf4_linear(*a) == aqnf4.AQNF4_ERR_ALIGNMENT
     assert lib.aqnf4_launch_count() == before
+    assert aqnf4.aqnf4_nf4_linear_workspace_size(4, 8, 96) == 0
