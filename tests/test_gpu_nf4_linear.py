@@ -113,3 +113,18 @@ def test_nf4_linear_rejects_bad_shapes():
     assert lib.aqnf4_nf4_linear(*a) == aqnf4.AQNF4_ERR_ALIGNMENT
     assert lib.aqnf4_launch_count() == before
     assert aqnf4.aqnf4_nf4_linear_workspace_size(4, 8, 96) == 0
+
+
+def test_split_k_workspace_sizes():
+    """The split rule on a 148-SM part (what the library assumes without a device):
+    enough splits for one wave, at least 8 steps of 64 each, none when the tiles fill it."""
+    if torch.cuda.is_available() and torch.cuda.get_device_properties(0).multi_processor_count != 148:
+        pytest.skip("sizes below are for 148 SMs")
+    # 11008 x 4096 layer, 128 tokens: 43 output tiles -> 148 // 43 = 3 splits
+    assert aqnf4.aqnf4_nf4_linear_workspace_size(128, 11008, 4096) == 3 * 128 * 11008 * 4
+    # 16 tokens, 1024 outputs, K 2048: 4 tiles -> 37, capped by 32 steps / 8 = 4
+    assert aqnf4.aqnf4_nf4_linear_workspace_size(16, 1024, 2048) == 4 * 16 * 1024 * 4
+    # K = 512: 8 steps cannot be split into two halves of >= 8 steps
+    assert aqnf4.aqnf4_nf4_linear_workspace_size(16, 1024, 512) == 0
+    # 4096 tokens x 11008: 16 x 43 = 688 tiles fill the GPU: no split
+    assert aqnf4.aqnf4_nf4_linear_workspace_size(4096, 11008, 4096) == 0
