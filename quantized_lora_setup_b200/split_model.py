@@ -70,6 +70,37 @@ class SplitModel:
         aqnf4.aqnf4_dequantize(st.packed, st.codes8, st.scales, None, L.numel, out, stream)
         return out
 
+    def linear(self, i: int, x: torch.Tensor, out_dtype: Optional[torch.dtype] = None,
+               stream=None) -> torch.Tensor:
+        """The forward product of layer i, y = x w^T, for x (M x K) in the layer's 16-bit
+        format: cuBLAS on the kept 16-bit weights, or the fused NF4-dequant tensor-core GEMM
+        (aqnf4_nf4_linear) on the NF4 + DQ storage.  A layer whose K is not a multiple of 64
+        (rows would not be whole NF4 blocks) is dequantized first and multiplied by cuBLAS."""
+        L = self.layers[i]
+        if len(L.shape) != 2:
+            raise ValueError("linear: the layer is not a matrix")
+        N, K = L.shape
+        out_dtype = out_dtype or x.dtype
+
+        def dense(w16):  # cuBLAS; a float32 result is summed in binary32 without 16-bit rounding
+            if out_dtype == torch.float32:
+                return torch.matmul(x.to(L.dtype).float(), w16.float().t())
+            return torch.matmul(x.to(L.dtype), w16.t()).to(out_dtype)
+
+        if L.kind == "fp16":
+            return dense(L.weight)
+        if K % 64 != 0 or x.dtype != L.dtype:
+            return dense(self.weight(i, stream=stream))
+        M = x.shape[0]
+        y = torch.empty((M, N), dtype=out_dtype if out_dtype == torch.float32 else x.dtype,
+                        device=x.device)
+        nbytes = aqnf4.aqnf4_nf4_linear_workspace_size(M, N, K)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=x.device) if nbytes else None
+        st = L.nf4
+        aqnf4.aqnf4_nf4_linear(x.contiguous(), st.packed, st.codes8, st.scales, N, y,
+                               stream=stream, workspace=ws)
+        return y.to(out_dtype)
+
     def memory_report(self) -> dict:
         fp16 = sum(L.held_bytes() for L in self.layers if L.kind == "fp16")
         nf4 = sum(L.held_bytes() for L in self.layers if L.kind == "nf4")

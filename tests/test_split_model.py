@@ -91,3 +91,38 @@ def test_materialize_ranks_by_dq_score_when_asked(cuda):
                     for w in weights], np.float32)
     assert model.kept == oracle.select_topk(rel, cost, budget)
     np.testing.assert_allclose([L.rel_err for L in model.layers], rel, rtol=1e-5)
+
+
+@pytest.mark.gpu
+def test_split_model_linear_matches_oracle(cuda):
+    """y = x w^T through the split model: the kept layer by cuBLAS on its 16-bit weights, an
+    NF4 layer by the fused tensor-core GEMM; both within the binary32 accumulation bound of
+    the oracle's binary64 product of what the layer holds."""
+    rng = np.random.default_rng(41)
+    shapes = [(256, 512), (384, 256), (130, 192)]
+    weights = [torch.from_numpy((rng.standard_normal(sh) * 0.02).astype(np.float32))
+               .to(torch.bfloat16).to(cuda) for sh in shapes]
+    cost = [aqnf4.aqnf4_cost_bytes(w.numel()) for w in weights]
+    # the largest layer's cost: the first-ranked layer always fits, not all of them can
+    model = split_model.materialize(weights, budget_bytes=max(cost))
+    kinds = {L.kind for L in model.layers}
+    assert kinds == {"fp16", "nf4"}
+    M = 96
+    for i, w in enumerate(weights):
+        N, K = shapes[i]
+        x = torch.from_numpy(rng.standard_normal((M, K)).astype(np.float32)).to(torch.bfloat16)
+        y = model.linear(i, x.to(cuda), out_dtype=torch.float32).double().cpu().numpy()
+        if model.layers[i].kind == "fp16":
+            w64 = w.double().cpu().numpy()
+        else:
+            w64 = model.weight(i).double().cpu().numpy()
+            packed, absmax, _ = oracle.quantize(synth.bits_u16(w.cpu()), oracle.BF16)
+            codes8, scales, _ = oracle.double_quant(absmax)
+            ref, _ = oracle.nf4_linear(synth.bits_u16(x).reshape(M, K), oracle.BF16, packed,
+                                       codes8, scales, N, oracle.BF16)
+            x64 = x.double().numpy()
+            assert np.allclose(x64 @ w64.T, ref, rtol=0, atol=1e-12)  # weight(i) is w_hat
+        x64 = x.double().numpy()
+        ref = x64 @ w64.T
+        bound = K * 2.0 ** -23 * (np.abs(x64) @ np.abs(w64).T) + 1e-30
+        assert np.all(np.abs(y - ref) <= bound), i
