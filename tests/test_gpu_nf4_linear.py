@@ -61,13 +61,14 @@ def test_nf4_linear_matches_oracle(cuda, dt, M, N, K):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("M,N,K", [(128, 11008, 4096), (16, 1024, 2048), (300, 512, 8192)])
-def test_nf4_linear_split_k_matches_oracle(cuda, M, N, K):
+def test_nf4_linear_split_k_matches_oracle(cuda, dt, M, N, K):
     """Few output tiles: K is split over several CTAs whose partials are added in order."""
     assert aqnf4.aqnf4_nf4_linear_workspace_size(M, N, K) > 0
-    x, packed, codes8, scales = _case(M, N, K, torch.bfloat16, seed=K + M)
-    ref, rabs = oracle.nf4_linear(synth.bits_u16(x).reshape(M, K), oracle.BF16, packed, codes8,
-                                  scales, N, oracle.BF16)
+    x, packed, codes8, scales = _case(M, N, K, dt, seed=K + M)
+    ref, rabs = oracle.nf4_linear(synth.bits_u16(x).reshape(M, K), DT[dt], packed, codes8,
+                                  scales, N, DT[dt])
     bound = K * 2.0 ** -23 * rabs + 1e-30
     y1 = _run(cuda, x, packed, codes8, scales, N, torch.float32)
     y2 = _run(cuda, x, packed, codes8, scales, N, torch.float32)
