@@ -9,13 +9,15 @@
 //
 // Blackwell structure.  One CTA (18 warps, one per SM) computes a 256 x 256 tile of y over
 // K in steps of 64, its roles specialised and coupled only through mbarriers:
-//   - warp 16 streams, by TMA and up to three steps ahead, the step's x tile (M x K, K
-//     contiguous; 128-byte-swizzled 256 x 64) and the matching 256-row x 32-byte slice of the
-//     packed codes;
-//   - warps 0-15 dequantize that slice into a 256 x 64 w_hat tile -- threads 2r and 2r + 1
-//     take the two halves of row n0 + r, one NF4 block per row and step (K is a multiple of
-//     64) -- in the same swizzled K-major layout, 16 bytes at a time, and arrive on the
-//     stage's barrier; the 8-bit constants and DQ scales come two steps ahead from global;
+//   - warp 16 streams, by TMA and up to kStagesA steps ahead, the step's x tile (M x K, K
+//     contiguous; 128-byte-swizzled 256 x 64);
+//   - warps 0-15 dequantize the step's 256-row slice of the layer into a 256 x 64 w_hat tile
+//     (one of kStagesB) -- threads 2r and 2r + 1 take the two halves of row n0 + r, one NF4
+//     block per row and step (K is a multiple of 64) -- in the same swizzled K-major layout,
+//     16 bytes at a time, and arrive on the tile's barrier.  Each thread loads its 16 bytes of
+//     packed codes, the block's 8-bit constant and its DQ scale from global memory three
+//     steps ahead into registers, so a w_hat tile can be rebuilt as soon as the tensor cores
+//     release it, without waiting for a copy;
 //   - warp 17 issues eight tcgen05.mma per step (M 128, N 256, K 16, bf16/f16 in, f32 out):
 //     each x row half against the same w_hat tile, into two TMEM accumulators that fill all
 //     512 columns, so every dequantized element feeds 256 rows of x; tcgen05.commit frees
@@ -33,14 +35,18 @@
 namespace aqnf4 {
 namespace {
 
-constexpr int kBM = 256, kBN = 256, kBK = 64, kStages = 3;  // two 128-row accumulators
+constexpr int kBM = 256, kBN = 256, kBK = 64;  // two 128-row accumulators
+// ring depths: x tiles (TMA) and w_hat tiles (dequantized); the dequantizing loop is unrolled
+// by kStagesB, so each of its steps works on a fixed tile and a fixed register set.  A fourth
+// x tile measured slower: the 231 KB of shared memory it takes leave too little of the SM's
+// on-chip memory to the L1 that serves the dequantizing warps' global loads.
+constexpr int kStagesA = 3, kStagesB = 3;
 constexpr int kDeqWarps = 16, kProducerWarp = 16, kMmaWarp = 17;
 constexpr int kGThreads = 32 * (kDeqWarps + 2);            // 576
 constexpr int kTileBytesA = kBM * kBK * 2;                  // 32 KB of x
 constexpr int kTileBytesB = kBN * kBK * 2;                  // 32 KB of w_hat
-constexpr int kTileBytesP = kBN * kBK / 2;                  // 8 KB of packed codes
-constexpr int kStageBytes = kTileBytesA + kTileBytesB + kTileBytesP;
-constexpr int kBarBase = kStages * kStageBytes;             // after the stages
+constexpr int kRingB = kStagesA * kTileBytesA;              // the w_hat ring follows the x ring
+constexpr int kBarBase = kRingB + kStagesB * kTileBytesB;   // after the rings
 constexpr int kFracOff = kBarBase + 256;                     // fl(c / 255) for c = 0..255
 constexpr int kGSmemBytes = kFracOff + 1024 + 1024;         // + alignment slack
 constexpr uint32_t kTmemCols = 512;  // two f32 accumulators of 256 columns: all of TMEM
@@ -134,17 +140,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 
 template <int DT>
 __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant__ CUtensorMap tmap_x,
-                                                           const __grid_constant__ CUtensorMap tmap_w,
                                                            const __grid_constant__ GParams p) {
   using F = Fmt<DT>;
   extern __shared__ uint8_t smem_raw[];
   // the swizzled tiles need 1024-byte alignment
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* full_a = reinterpret_cast<uint64_t*>(smem + kBarBase);
-  uint64_t* full_b = full_a + kStages;
-  uint64_t* empty = full_b + kStages;
-  uint64_t* accum = empty + kStages;
+  uint64_t* full_a = reinterpret_cast<uint64_t*>(smem + kBarBase);  // x tile landed
+  uint64_t* empty_a = full_a + kStagesA;                            // x tile consumed
+  uint64_t* full_b = empty_a + kStagesA;                            // w_hat tile written
+  uint64_t* empty_b = full_b + kStagesB;                            // w_hat tile consumed
+  uint64_t* accum = empty_b + kStagesB;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accum + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   float* frac = reinterpret_cast<float*>(smem + kFracOff);
@@ -160,10 +166,13 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
   const bool lower_half = m0 + 128 < p.M;  // the tile's second 128 rows hold any of x
 
   if (t == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kStagesA; ++s) {
       mbar_init(smem_addr(full_a + s), 1);
+      mbar_init(smem_addr(empty_a + s), 1);
+    }
+    for (int s = 0; s < kStagesB; ++s) {
       mbar_init(smem_addr(full_b + s), 32 * kDeqWarps);
-      mbar_init(smem_addr(empty + s), 1);
+      mbar_init(smem_addr(empty_b + s), 1);
     }
     mbar_init(smem_addr(accum), 1);
     *abort_flag = 0;
@@ -181,42 +190,36 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  int64_t last_kt[kStages];  // producer: the last step copied into each stage (-1: none)
-#pragma unroll
-  for (int s = 0; s < kStages; ++s) last_kt[s] = -1;
+  int64_t issued = 0;  // producer: x copies issued (step i went to tile i mod kStagesA)
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
       for (int64_t i = 0; i < nk && !*abort_flag; ++i) {
-        const int64_t kt = kt0 + i;
-        const int s = static_cast<int>(i % kStages);
-        const uint32_t use = static_cast<uint32_t>(i / kStages);
-        if (i >= kStages && !mbar_wait_bounded(smem_addr(empty + s), (use - 1) & 1)) {
+        const int s = static_cast<int>(i % kStagesA);
+        const uint32_t use = static_cast<uint32_t>(i / kStagesA);
+        if (i >= kStagesA && !mbar_wait_bounded(smem_addr(empty_a + s), (use - 1) & 1)) {
           *abort_flag = 1;
           break;
         }
-        uint8_t* st = smem + s * kStageBytes;
-        mbar_arrive_expect_tx(smem_addr(full_a + s), kTileBytesA + kTileBytesP);
-        tma_load_2d(smem_addr(st), &tmap_x, static_cast<int>(kt * kBK), static_cast<int>(m0),
+        mbar_arrive_expect_tx(smem_addr(full_a + s), kTileBytesA);
+        tma_load_2d(smem_addr(smem + s * kTileBytesA), &tmap_x,
+                    static_cast<int>((kt0 + i) * kBK), static_cast<int>(m0),
                     smem_addr(full_a + s));
-        tma_load_2d(smem_addr(st + kTileBytesA + kTileBytesB), &tmap_w,
-                    static_cast<int>(kt * (kBK / 2)), static_cast<int>(n0), smem_addr(full_a + s));
-        last_kt[s] = i;
+        issued = i + 1;
       }
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
       for (int64_t i = 0; i < nk && !*abort_flag; ++i) {
-        const int s = static_cast<int>(i % kStages);
-        const uint32_t par = static_cast<uint32_t>(i / kStages) & 1;
-        if (!mbar_wait_bounded(smem_addr(full_a + s), par) ||
-            !mbar_wait_bounded(smem_addr(full_b + s), par)) {
+        const int sa = static_cast<int>(i % kStagesA), sb = static_cast<int>(i % kStagesB);
+        if (!mbar_wait_bounded(smem_addr(full_a + sa), static_cast<uint32_t>(i / kStagesA) & 1) ||
+            !mbar_wait_bounded(smem_addr(full_b + sb), static_cast<uint32_t>(i / kStagesB) & 1)) {
           *abort_flag = 1;
           break;
         }
         tc_fence_after();
-        const uint32_t a0 = smem_addr(smem + s * kStageBytes);
-        const uint32_t b0 = a0 + kTileBytesA;
+        const uint32_t a0 = smem_addr(smem + sa * kTileBytesA);
+        const uint32_t b0 = smem_addr(smem + kRingB + sb * kTileBytesB);
 #pragma unroll
         for (int j = 0; j < kBK / 16; ++j) {  // K = 16 per MMA: 32 bytes along the swizzled row
           // rows 0..127 of x into columns 0..255 of TMEM, rows 128..255 into 256..511; both
@@ -227,49 +230,40 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
             umma_f16(tmem + kBN, sw128_desc(a0 + 128 * 128 + 32 * j), sw128_desc(b0 + 32 * j),
                      idesc<DT>(), (i > 0 || j > 0) ? 1u : 0u);
         }
-        umma_commit(smem_addr(empty + s));
+        umma_commit(smem_addr(empty_a + sa));  // each arrives once the MMAs above have finished
+        umma_commit(smem_addr(empty_b + sb));
       }
       umma_commit(smem_addr(accum));  // arrives once every MMA issued above has finished
     }
   } else {
     // ---- dequantizing warps: threads 2r and 2r + 1 own the two halves of row n0 + r of the
-    // w_hat tile.  The packed codes arrive by TMA with x; the 8-bit constant and the DQ scale
-    // of steps kt + 1 and kt + 2 are loaded from global memory while step kt is worked on.
+    // w_hat tile.  Step i's 16 bytes of packed codes, 8-bit constant and DQ scale are loaded
+    // from global memory while steps i - 3 .. i - 1 are worked on; the loop is unrolled by
+    // kStagesB (= 3), so step i + u always uses w_hat tile u and register set u.
     const float tab_level = p.level[lane & 15];  // lanes 16..31 mirror 0..15
     const int r = t >> 1, hf = t & 1;
     const int64_t n = n0 + r;
     const bool row_ok = n < p.N;
-    // (code8, scale) of steps kt, kt + 1, kt + 2, rotated through registers
-    uint32_t c8_0 = 0, c8_1 = 0, c8_2 = 0;
-    float sc_0 = 0.0f, sc_1 = 0.0f, sc_2 = 0.0f;
-    auto fetch = [&](int64_t kt, uint32_t& c, float& s8) {
+    const uint8_t* prow = p.packed + n * (p.K / 2) + hf * 16;
+    auto fetch = [&](int64_t kt, uint4& pk, uint32_t& c, float& s8) {
       if (row_ok && kt < kt1) {
         const int64_t b = n * kb + kt;
+        pk = __ldg(reinterpret_cast<const uint4*>(prow + kt * (kBK / 2)));
         c = __ldg(p.codes8 + b);
         s8 = __ldg(p.scales + (b >> 8));
       }
     };
-    fetch(kt0, c8_0, sc_0);
-    fetch(kt0 + 1, c8_1, sc_1);
-    for (int64_t i = 0; i < nk; ++i) {
-      const int64_t kt = kt0 + i;
-      const int s = static_cast<int>(i % kStages);
-      const uint32_t use = static_cast<uint32_t>(i / kStages);
-      c8_2 = 0;
-      sc_2 = 0.0f;
-      fetch(kt + 2, c8_2, sc_2);
-      bool ok = true;
-      if (i >= kStages) ok = mbar_wait_bounded(smem_addr(empty + s), (use - 1) & 1);
-      ok = ok && mbar_wait_bounded(smem_addr(full_a + s), use & 1);  // packed codes landed
+    // one step into w_hat tile u; false when the pipeline has been aborted
+    auto dequant = [&](int64_t i, int u, const uint4& pk, uint32_t c8, float sc) -> bool {
+      bool ok = i < kStagesB ||
+                mbar_wait_bounded(smem_addr(empty_b + u), static_cast<uint32_t>(i / kStagesB - 1) & 1);
       if (!ok) *abort_flag = 1;
-      if (__any_sync(kFull, *abort_flag != 0)) break;  // warp-uniform exit (shuffles below)
-      uint8_t* st = smem + s * kStageBytes;
-      const uint4 pk = *reinterpret_cast<const uint4*>(st + kTileBytesA + kTileBytesB + r * 32 + hf * 16);
-      // a zero constant (also for rows past N, whose codes are the copy's zero fill) gives 0
-      const float ap = row_ok ? __fmul_rn(frac[c8_0], sc_0) : 0.0f;
+      if (__any_sync(kFull, *abort_flag != 0)) return false;  // warp-uniform (shuffles below)
+      // a zero constant (also for rows past N) gives 0
+      const float ap = row_ok ? __fmul_rn(frac[c8], sc) : 0.0f;
       const f32x2 a2 = pair(ap, ap);
       const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
-      uint8_t* rowb = st + kTileBytesA + (r >> 3) * 1024 + (r & 7) * 128;
+      uint8_t* rowb = smem + kRingB + u * kTileBytesB + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
         const uint32_t w = words[jj];
@@ -286,11 +280,23 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
         *reinterpret_cast<uint4*>(rowb + ((j ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
       }
       fence_proxy_async_smem();  // the tensor cores read this tile through the async proxy
-      mbar_arrive(smem_addr(full_b + s));
-      c8_0 = c8_1;
-      sc_0 = sc_1;
-      c8_1 = c8_2;
-      sc_1 = sc_2;
+      mbar_arrive(smem_addr(full_b + u));
+      return true;
+    };
+    static_assert(kStagesB == 3, "the dequantizing loop below is unrolled by three");
+    uint4 pk0 = make_uint4(0, 0, 0, 0), pk1 = pk0, pk2 = pk0;
+    uint32_t c0 = 0, c1 = 0, c2 = 0;
+    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f;
+    fetch(kt0, pk0, c0, s0);
+    fetch(kt0 + 1, pk1, c1, s1);
+    fetch(kt0 + 2, pk2, c2, s2);
+    for (int64_t i = 0; i < nk; i += 3) {
+      if (!dequant(i, 0, pk0, c0, s0)) break;
+      fetch(kt0 + i + 3, pk0, c0, s0);
+      if (i + 1 >= nk || !dequant(i + 1, 1, pk1, c1, s1)) break;
+      fetch(kt0 + i + 4, pk1, c1, s1);
+      if (i + 2 >= nk || !dequant(i + 2, 2, pk2, c2, s2)) break;
+      fetch(kt0 + i + 5, pk2, c2, s2);
     }
   }
 
@@ -341,10 +347,11 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
     }
   }
   if (warp == kProducerWarp && lane == 0 && failed) {
-    // let every copy issued land before the shared memory goes away
-    for (int s = 0; s < kStages; ++s)
-      if (last_kt[s] >= 0)
-        mbar_wait_bounded(smem_addr(full_a + s), static_cast<uint32_t>(last_kt[s] / kStages) & 1);
+    // let every copy issued land before the shared memory goes away: tile s last received
+    // step s + kStagesA * ((issued - 1 - s) / kStagesA)
+    for (int s = 0; s < kStagesA && s < issued; ++s)
+      mbar_wait_bounded(smem_addr(full_a + s),
+                        static_cast<uint32_t>((issued - 1 - s) / kStagesA) & 1);
   }
   tc_fence_before();
   __syncthreads();
@@ -406,15 +413,14 @@ EncodeTiledFn encode_tiled() {
 }
 
 template <int DT>
-cudaError_t launch_gemm(const CUtensorMap& map, const CUtensorMap& wmap, const GParams& p,
-                        cudaStream_t stream) {
+cudaError_t launch_gemm(const CUtensorMap& map, const GParams& p, cudaStream_t stream) {
   auto kern = k_nf4_gemm<DT>;
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmemBytes);
   if (err != cudaSuccess) return err;
   const dim3 grid(static_cast<unsigned>((p.N + kBN - 1) / kBN),
                   static_cast<unsigned>((p.M + kBM - 1) / kBM), static_cast<unsigned>(p.splits));
-  kern<<<grid, kGThreads, kGSmemBytes, stream>>>(map, wmap, p);
+  kern<<<grid, kGThreads, kGSmemBytes, stream>>>(map, p);
   count_launches(1);
   if (p.splits > 1) {
     const int64_t mn = p.M * p.N;
@@ -467,15 +473,6 @@ extern "C" aqnf4_status aqnf4_nf4_linear(const void* x, int32_t dtype, int64_t M
              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return AQNF4_ERR_INVALID_ARG;
-  // packed codes as an N x K/2 byte matrix: a 256-row x 32-byte box is one step's slice
-  CUtensorMap wmap;
-  const cuuint64_t wdims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(N)};
-  const cuuint64_t wstrides[1] = {static_cast<cuuint64_t>(K / 2)};
-  const cuuint32_t wbox[2] = {kBK / 2, kBN};
-  if (encode(&wmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(packed), wdims,
-             wstrides, wbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return AQNF4_ERR_INVALID_ARG;
   GParams p;
   p.packed = packed;
   p.codes8 = codes8;
@@ -492,7 +489,7 @@ extern "C" aqnf4_status aqnf4_nf4_linear(const void* x, int32_t dtype, int64_t M
     p.splits = 1;  // no room for the partial sums: one CTA per output tile
   p.flag = dev_flag;
   for (int i = 0; i < 16; ++i) p.level[i] = tb->level[i];
-  const cudaError_t err = dtype == AQNF4_BF16 ? launch_gemm<AQNF4_BF16>(map, wmap, p, stream)
-                                              : launch_gemm<AQNF4_F16>(map, wmap, p, stream);
+  const cudaError_t err = dtype == AQNF4_BF16 ? launch_gemm<AQNF4_BF16>(map, p, stream)
+                                              : launch_gemm<AQNF4_F16>(map, p, stream);
   return err == cudaSuccess ? AQNF4_OK : AQNF4_ERR_CUDA;
 }
