@@ -45,7 +45,7 @@ constexpr int kThreads = kDqBlock / kBpt;  // a CTA covers one tile (= one DQ bl
 constexpr int kWarps = kThreads / 32;
 // chunk loop of the coding pass unrolled by 2: smaller code, slightly faster than full unroll
 constexpr int kP2Unroll = 2;
-constexpr int kCtasPerSm = 4;  // 44 KB of shared memory and 128 registers per thread, no spills
+constexpr int kCtasPerSm = 5;  // 44 KB of shared memory and <= 102 registers per thread, no spills
 constexpr int kMaxLayersPerLaunch = 384;
 
 // The coding loop keeps each code as c = bits(2^23 + slot) + (v > mid) = kCodeBias + code,
