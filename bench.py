@@ -43,6 +43,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dequant", action="store_true")
+    ap.add_argument("--no-dequant-sweep", action="store_true",
+                    help="skip the dequantize sweep (packed 1 MB .. 4 GB and the named shapes)")
     ap.add_argument("--no-nf4-linear", action="store_true",
                     help="skip the fused NF4-dequant GEMM measurement")
     ap.add_argument("--only-nf4-linear", action="store_true",
@@ -373,6 +375,8 @@ def run_native(args):
 
     if not args.no_dequant:
         result["dequant"] = bench_dequant(dev, stream, peak)
+    if not args.no_dequant and not args.no_dequant_sweep:
+        result["dequant_sweep"] = bench_dequant_sweep(dev, stream, peak)
 
     if world == 1:
         result["select_blocks"] = bench_select_blocks(wl, se, sw, cost, budget, dev, stream)
@@ -685,14 +689,68 @@ def bench_dequant(dev, stream, peak):
     b.record(stream)
     torch.cuda.synchronize(dev)
     ms = a.elapsed_time(b) / reps
-    nb = (n + 63) // 64
-    alg = n // 2 + nb + 4 * ((nb + 255) // 256) + 2 * n
+    alg = dequant_alg_bytes(n)
     gbs = alg / (ms / 1e3) / 1e9
     return {"shape": f"{rows}x{cols}", "ms_per_launch": ms, "value": gbs, "unit": "GB/s",
             "out_gbs": 2 * n / (ms / 1e3) / 1e9,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
                          "frac": gbs / peak, "traffic": None, "kernel": "k_dequant",
                          "alg_bytes_per_launch": alg}}
+
+
+def dequant_alg_bytes(n):
+    """Bytes one dequantize of n elements must move: packed codes, 8-bit constants and DQ
+    scales in, 16-bit values out."""
+    nb = (n + 63) // 64
+    return n // 2 + nb + 4 * ((nb + 255) // 256) + 2 * n
+
+
+def bench_dequant_sweep(dev, stream, peak, reps=9):
+    """NF4 + DQ -> bf16 over packed sizes 1 MB .. 4 GB (x2) and the named matrix shapes,
+    each stored from an N(0, 0.02) bf16 matrix by the scoring pass.  Before every launch L2
+    is flushed: a 256 MB write, then a read of another 256 MB so that the written lines
+    are back in DRAM before the timed launch starts.  Each launch is timed alone with
+    events on the launching stream and the median is reported, so every size is measured
+    from DRAM with a clean L2."""
+    import torch
+
+    from quantized_lora_setup_b200 import aqnf4, synth
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    clean = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    cases = [("packed_%dMB" % (1 << e), 4096, (2 << 20 << e) // 4096) for e in range(13)]
+    cases += [("%dx%d" % rc, rc[1], rc[0]) for rc in (synth.DEQUANT_SHAPES[0],
+                                                      synth.DEQUANT_SHAPES[-1])]
+    points = []
+    for name, cols, rows in cases:
+        n = rows * cols
+        w = synth.normal_matrix_device(rows, cols, seed=77, device=dev)
+        st = aqnf4.NF4Storage(n, dev)
+        aqnf4.score_layers([w.reshape(-1)], [st], stream=stream)
+        del w
+        out = torch.empty(n, dtype=torch.bfloat16, device=dev)
+        aqnf4.aqnf4_dequantize(st.packed, st.codes8, st.scales, None, n, out, stream)
+        times = []
+        for _ in range(reps):
+            with torch.cuda.stream(stream):
+                flush.fill_(1)
+                clean.sum()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            aqnf4.aqnf4_dequantize(st.packed, st.codes8, st.scales, None, n, out, stream)
+            b.record(stream)
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        ms = sorted(times)[reps // 2]
+        alg = dequant_alg_bytes(n)
+        gbs = alg / (ms / 1e3) / 1e9
+        points.append({"case": name, "packed_bytes": n // 2, "elements": n,
+                       "us": ms * 1e3, "value": gbs, "frac": gbs / peak})
+        del st, out
+    torch.cuda.empty_cache()
+    return {"unit": "GB/s", "peak": peak, "kernel": "k_dequant", "dtype_out": "bfloat16",
+            "l2": "flushed before every launch (256 MB write, then 256 MB read); median of %d"
+                  % reps,
+            "points": points}
 
 
 def bench_e2e(args, weights, step, sel, kout, dev, stream, world, total_weight_bytes, L):

@@ -6,7 +6,7 @@ oracle then recomputes a sample of layers one by one (first, middle, last, and o
 each value distribution): packed codes, DQ bytes and scales must be bit-exact and the
 scores within 1e-5.  The selection at every budget must equal the oracle's selection on
 the same score vector.  The standalone dequantization of a 28672x8192 matrix is checked
-on DQ-block-aligned slices.
+on DQ-block-aligned slices, and one layer of more than 2^32 elements on sampled tiles.
 """
 from concurrent.futures import ThreadPoolExecutor
 
@@ -111,3 +111,38 @@ def test_full_model_dq_score_sampled_layers(cuda):
         assert se[i].item() == pytest.approx(ose, rel=RTOL), i
         assert sw[i].item() == pytest.approx(osw, rel=RTOL), i
         assert rel[i].item() == pytest.approx(orel, rel=RTOL), i
+
+
+def test_single_layer_beyond_2_32_elements(cuda):
+    """One bf16 layer of 2^33 + 3 * 16384 + 100 elements: element, byte and block offsets
+    pass 2^31 and 2^32, and the last DQ tile (100 elements, two blocks, the second short) is
+    ragged.  A DQ tile's storage depends only on its own 16384 elements, so the oracle,
+    run on each sampled tile alone, fixes its packed codes, DQ bytes and scale bit for bit,
+    and the standalone dequantization of the same tiles."""
+    tile = 16384
+    n = (1 << 33) + 3 * tile + 100
+    w = torch.empty(n, dtype=torch.bfloat16, device=cuda)
+    g = torch.Generator(device=cuda)
+    g.manual_seed(11)
+    step = 1 << 28
+    for s in range(0, n, step):
+        e = min(n, s + step)
+        w[s:e] = (torch.randn(e - s, generator=g, device=cuda) * 0.02).to(torch.bfloat16)
+    st = aqnf4.NF4Storage(n, cuda)
+    _, _, rel = aqnf4.score_layers([w], [st])
+    out = aqnf4.dequantize(st.packed, n, torch.bfloat16, codes8=st.codes8, scales=st.scales)
+    torch.cuda.synchronize()
+    assert 0.005 < rel.item() < 0.15
+    ntiles = (n + tile - 1) // tile
+    t31, t32 = (1 << 31) // tile, (1 << 32) // tile
+    for t in (0, 1, t31 - 1, t31, t32 - 1, t32, ntiles - 2, ntiles - 1):
+        e0, e1 = t * tile, min(n, (t + 1) * tile)
+        b0, b1 = e0 // 64, (e1 + 63) // 64
+        bits = synth.bits_u16(w[e0:e1].cpu())
+        op, oa, _ = oracle.quantize(bits, oracle.BF16)
+        oc, osc, _ = oracle.double_quant(oa)
+        assert np.array_equal(st.packed[e0 // 2:(e1 + 1) // 2].cpu().numpy(), op), t
+        assert np.array_equal(st.codes8[b0:b1].cpu().numpy(), oc), t
+        assert st.scales[t].cpu().numpy().view(np.uint32) == osc.view(np.uint32)[0], t
+        ref = oracle.dequantize(op, e1 - e0, oracle.BF16, codes8=oc, scales=osc)
+        assert np.array_equal(synth.bits_u16(out[e0:e1].cpu()), ref), t

@@ -44,7 +44,8 @@ def _run(cuda, x, packed, codes8, scales, N, out_dtype, split=True):
 @pytest.mark.gpu
 @pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("M,N,K", [(128, 128, 64), (1, 1, 64), (200, 300, 256),
-                                   (256, 384, 4096), (130, 129, 192)])
+                                   (256, 384, 4096), (130, 129, 192), (64, 100, 128),
+                                   (70, 260, 320)])
 def test_nf4_linear_matches_oracle(cuda, dt, M, N, K):
     x, packed, codes8, scales = _case(M, N, K, dt, seed=M + N + K)
     ref, rabs = oracle.nf4_linear(synth.bits_u16(x).reshape(M, K), DT[dt], packed, codes8,
