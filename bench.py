@@ -58,6 +58,13 @@ def parse_args():
                     help="comma-separated workloads also timed (1 GPU only; '' to skip)")
     ap.add_argument("--max-layers", type=int, default=0,
                     help="use only the first N layers (small cases for profiling)")
+    ap.add_argument("--protocol", action="store_true",
+                    help="also run the source pages' timing protocol: two identical arms of "
+                         ">= 2 s each (noise floor); the CPU baseline is also timed on one "
+                         "thread")
+    ap.add_argument("--sessions", type=int, default=1,
+                    help="run this many whole sessions (separate processes, each with "
+                         "--protocol) and report their median and spread (1 GPU only)")
     return ap.parse_args()
 
 
@@ -373,6 +380,10 @@ def run_native(args):
         "selected": {"k": k_sel, "of": L},
     }
 
+    if args.protocol:
+        result["protocol"] = bench_protocol(step, dev, stream, world, total_weight_bytes,
+                                            elapsed_ms / K)
+
     if not args.no_dequant:
         result["dequant"] = bench_dequant(dev, stream, peak)
     if not args.no_dequant and not args.no_dequant_sweep:
@@ -407,6 +418,10 @@ def run_native(args):
             "sample": f"{len(sample)} slices of up to {per_thread} elements from the first "
                       f"{len(sample)} layers ({elems} weights), quantize + DQ + error, one "
                       f"thread per slice"}
+        if args.protocol:  # the pages' second oracle timing: one slice on one thread
+            t0 = time.perf_counter()
+            one = oracle_pass(sample[:1])
+            result["cpu_baseline"]["single_thread"] = 2 * one / (time.perf_counter() - t0) / 1e9
 
     extras = [w for w in args.extra_workloads.split(",") if w and w != args.workload]
     if world == 1 and extras:
@@ -788,10 +803,93 @@ def bench_e2e(args, weights, step, sel, kout, dev, stream, world, total_weight_b
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4 + 4 * L, "steps": steps}
 
 
+def bench_protocol(step, dev, stream, world, total_weight_bytes, ms_per_step,
+                   min_seconds=2.0):
+    """The source pages' timing rules for the scoring step: the same step is run as two
+    arms, "a" and "b", each back to back for at least `min_seconds` of device time (a fixed
+    duration, not a fixed count), timed with CUDA events in chunks of about 0.25 s.  With
+    several ranks each chunk's time is the maximum over ranks, so every rank takes the same
+    number of chunks.  The relative gap between the arms is the noise floor."""
+    import torch
+    import torch.distributed as dist
+
+    chunk = max(1, int(250.0 / max(ms_per_step, 1e-3)))
+    arms = {}
+    for arm in ("a", "b"):
+        total_ms, steps = 0.0, 0
+        while total_ms < min_seconds * 1e3:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            a.record(stream)
+            for _ in range(chunk):
+                step()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            ms = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+            if world > 1:
+                dist.all_reduce(ms, op=dist.ReduceOp.MAX)
+            total_ms += float(ms.item())
+            steps += chunk
+        arms[arm] = {"steps": steps, "seconds": total_ms / 1e3,
+                     "value": total_weight_bytes * steps / (total_ms / 1e3) / 1e9}
+    va, vb = arms["a"]["value"], arms["b"]["value"]
+    return {"min_seconds_per_arm": min_seconds, "unit": UNIT, "arms": arms,
+            "noise_floor": abs(va - vb) / ((va + vb) / 2)}
+
+
+def session_child_argv(argv):
+    """The command line of one session: this one without --sessions, with --protocol."""
+    child, i = [], 0
+    while i < len(argv):
+        if argv[i] == "--sessions":
+            i += 2
+            continue
+        if not argv[i].startswith("--sessions="):
+            child.append(argv[i])
+        i += 1
+    if "--protocol" not in child:
+        child.append("--protocol")
+    return child
+
+
+def run_sessions(args):
+    """Whole sessions as separate processes (each with --protocol); prints the median
+    session's line with the per-session values, their median and their spread."""
+    import subprocess
+
+    child = session_child_argv(sys.argv[1:])
+    lines = []
+    for _ in range(args.sessions):
+        out = subprocess.run([sys.executable, os.path.abspath(__file__)] + child,
+                             capture_output=True, text=True)
+        if out.returncode != 0:
+            sys.stderr.write(out.stdout[-2000:] + out.stderr[-4000:])
+            return out.returncode
+        lines.append(json.loads(out.stdout.strip().splitlines()[-1]))
+    vals = [d["value"] for d in lines]
+    med = statistics.median(vals)
+    pick = min(range(len(lines)), key=lambda j: abs(vals[j] - med))
+    arm_vals = [d["protocol"]["arms"][a]["value"] for d in lines for a in ("a", "b")]
+    res = dict(lines[pick])
+    res["sessions"] = {
+        "n": len(lines), "values": vals, "median": med,
+        "spread": (max(vals) - min(vals)) / med,
+        "protocol_arm_values": arm_vals,
+        "protocol_arm_median": statistics.median(arm_vals),
+        "protocol_arm_spread": (max(arm_vals) - min(arm_vals)) / statistics.median(arm_vals),
+        "noise_floors": [d["protocol"]["noise_floor"] for d in lines]}
+    print(json.dumps(res), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.sessions > 1:
+        if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+            raise SystemExit("--sessions runs separate single-GPU processes; not under torchrun")
+        return run_sessions(args)
     if args.only_nf4_linear:
         return run_only_nf4_linear(args)
     return run_native(args)
