@@ -68,6 +68,9 @@ def parse_args():
     return ap.parse_args()
 
 
+L2_BYTES = 126 << 20
+
+
 def host_threads() -> int:
     try:
         n = len(os.sched_getaffinity(0))
@@ -366,7 +369,9 @@ def run_native(args):
         "config": {
             "workload": workload_desc(wl), "layers": L, "weight_bytes": total_weight_bytes,
             "budget_bytes": budget, "k_cap": wl.k_cap,
-            "l2": "inputs larger than L2 (weights read once per step, no flush needed)",
+            "l2": "inputs larger than L2 (weights read once per step, no flush needed)"
+            if total_weight_bytes >= 2 * L2_BYTES else
+            "L2-resident: the working set is below twice the 126 MB L2 (reported as such)",
             "parallelism": f"layers split over {world} rank(s) by LPT; scores all-gathered"
             if world > 1 else "single GPU",
             "outputs": "packed NF4 + 8-bit DQ codes + fp32 DQ scales + per-layer scores",
