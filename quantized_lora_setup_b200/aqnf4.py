@@ -134,6 +134,31 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(int(stream))
 
 
+def _req(t: Optional[torch.Tensor], name: str, dtypes, min_numel: int = 0,
+         optional: bool = False) -> None:
+    """Checks the C ABI cannot make on bare pointers, done before any launch: a CUDA tensor,
+    contiguous, of an accepted dtype (None: any; the library checks 16-bit formats itself)
+    and holding at least min_numel elements.  Raises ValueError."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name}: required")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected one of {dtypes}")
+    if t.numel() < min_numel:
+        raise ValueError(f"{name}: {t.numel()} elements, at least {min_numel} needed")
+
+
+def _storage_sizes(n: int):
+    """(packed bytes, blocks, DQ scales) of n weights."""
+    nb = (n + BLOCK - 1) // BLOCK
+    return (n + 1) // 2, nb, (nb + DQ_BLOCK - 1) // DQ_BLOCK
+
+
 def dtype_code(dtype: torch.dtype) -> int:
     try:
         return _DT_CODE[dtype]
@@ -156,6 +181,11 @@ def aqnf4_codebook(p_max: float = 0.0):
 
 def aqnf4_quantize(w: torch.Tensor, packed: Optional[torch.Tensor], absmax: Optional[torch.Tensor],
                    dev_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    npk, nb, _ = _storage_sizes(w.numel())
+    _req(w, "w", None)
+    _req(packed, "packed", (torch.uint8,), npk, optional=True)
+    _req(absmax, "absmax", (torch.float32,), nb, optional=True)
+    _req(dev_flag, "dev_flag", (torch.int32,), 1, optional=True)
     _check(library().aqnf4_quantize(_ptr(w), dtype_code(w.dtype), w.numel(), _ptr(packed),
                                     _ptr(absmax), _ptr(dev_flag), _stream(stream)),
            "aqnf4_quantize")
@@ -163,6 +193,11 @@ def aqnf4_quantize(w: torch.Tensor, packed: Optional[torch.Tensor], absmax: Opti
 
 def aqnf4_double_quant(absmax: torch.Tensor, codes8: torch.Tensor, scales: torch.Tensor,
                        dev_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    nb = absmax.numel()
+    _req(absmax, "absmax", (torch.float32,))
+    _req(codes8, "codes8", (torch.uint8,), nb)
+    _req(scales, "scales", (torch.float32,), (nb + DQ_BLOCK - 1) // DQ_BLOCK)
+    _req(dev_flag, "dev_flag", (torch.int32,), 1, optional=True)
     _check(library().aqnf4_double_quant(_ptr(absmax), absmax.numel(), _ptr(codes8), _ptr(scales),
                                         _ptr(dev_flag), _stream(stream)), "aqnf4_double_quant")
 
@@ -170,6 +205,12 @@ def aqnf4_double_quant(absmax: torch.Tensor, codes8: torch.Tensor, scales: torch
 def aqnf4_dequantize(packed: torch.Tensor, codes8: Optional[torch.Tensor],
                      scales: Optional[torch.Tensor], absmax: Optional[torch.Tensor], n: int,
                      out: torch.Tensor, stream=None) -> None:
+    npk, nb, nsc = _storage_sizes(n)
+    _req(packed, "packed", (torch.uint8,), npk)
+    _req(codes8, "codes8", (torch.uint8,), nb, optional=True)
+    _req(scales, "scales", (torch.float32,), nsc, optional=True)
+    _req(absmax, "absmax", (torch.float32,), nb, optional=True)
+    _req(out, "out", None, n)
     _check(library().aqnf4_dequantize(_ptr(packed), _ptr(codes8), _ptr(scales), _ptr(absmax), n,
                                       dtype_code(out.dtype), _ptr(out), _stream(stream)),
            "aqnf4_dequantize")
@@ -181,6 +222,11 @@ def make_layers(layers: Sequence[dict]):
     arr = (aqnf4_layer * len(layers))()
     for i, d in enumerate(layers):
         w = d["w"]
+        _req(w, f"layers[{i}].w", None)
+        npk, nb, nsc = _storage_sizes(w.numel())
+        for key, dt, need in (("packed", torch.uint8, npk), ("absmax", torch.float32, nb),
+                              ("codes8", torch.uint8, nb), ("scales", torch.float32, nsc)):
+            _req(d.get(key), f"layers[{i}].{key}", (dt,), need, optional=True)
         arr[i].w = w.data_ptr()
         arr[i].numel = w.numel()
         arr[i].dtype = dtype_code(w.dtype)
@@ -196,10 +242,19 @@ def aqnf4_workspace_size(layers) -> int:
     return int(library().aqnf4_workspace_size(arr, len(arr)))
 
 
+def _check_outputs(L, sq_err, sq_w, rel_err, dev_flag):
+    _req(sq_err, "sq_err", (torch.float64,), L, optional=True)
+    _req(sq_w, "sq_w", (torch.float64,), L, optional=True)
+    _req(rel_err, "rel_err", (torch.float32,), L, optional=True)
+    _req(dev_flag, "dev_flag", (torch.int32,), 1, optional=True)
+
+
 def aqnf4_layer_error(layers, workspace: torch.Tensor, sq_err: Optional[torch.Tensor],
                       sq_w: Optional[torch.Tensor], rel_err: Optional[torch.Tensor],
                       dev_flag: Optional[torch.Tensor] = None, stream=None) -> None:
     arr = layers if isinstance(layers, ctypes.Array) else make_layers(layers)
+    _req(workspace, "workspace", None)
+    _check_outputs(len(arr), sq_err, sq_w, rel_err, dev_flag)
     nbytes = workspace.numel() * workspace.element_size()
     _check(library().aqnf4_layer_error(arr, len(arr), _ptr(workspace), nbytes, _ptr(sq_err),
                                        _ptr(sq_w), _ptr(rel_err), _ptr(dev_flag),
@@ -211,6 +266,7 @@ def aqnf4_layer_error_noalloc(layers, sq_err: Optional[torch.Tensor],
                               dev_flag: Optional[torch.Tensor] = None, stream=None) -> None:
     """aqnf4_layer_error with the library's built-in scratch instead of a workspace."""
     arr = layers if isinstance(layers, ctypes.Array) else make_layers(layers)
+    _check_outputs(len(arr), sq_err, sq_w, rel_err, dev_flag)
     _check(library().aqnf4_layer_error_noalloc(arr, len(arr), _ptr(sq_err), _ptr(sq_w),
                                                _ptr(rel_err), _ptr(dev_flag), _stream(stream)),
            "aqnf4_layer_error_noalloc")
@@ -219,6 +275,11 @@ def aqnf4_layer_error_noalloc(layers, sq_err: Optional[torch.Tensor],
 def aqnf4_select_topk(rel_err: torch.Tensor, cost_bytes: torch.Tensor, budget_bytes: int,
                       k_cap: int, sel_idx: torch.Tensor, k_out: torch.Tensor,
                       stream=None) -> None:
+    L = rel_err.numel()
+    _req(rel_err, "rel_err", (torch.float32,))
+    _req(cost_bytes, "cost_bytes", (torch.int64,), L)
+    _req(sel_idx, "sel_idx", (torch.int32,), L)
+    _req(k_out, "k_out", (torch.int32,), 1)
     _check(library().aqnf4_select_topk(_ptr(rel_err), _ptr(cost_bytes), rel_err.numel(),
                                        int(budget_bytes), int(k_cap), _ptr(sel_idx), _ptr(k_out),
                                        _stream(stream)), "aqnf4_select_topk")
@@ -236,10 +297,20 @@ def aqnf4_nf4_linear(x: torch.Tensor, packed: torch.Tensor, codes8: torch.Tensor
                      workspace: Optional[torch.Tensor] = None) -> None:
     """y (M x N) = x (M x K) w_hat^T for the N x K layer stored as packed + codes8 + scales;
     y may be float32 or x's dtype.  workspace: see aqnf4_nf4_linear_workspace_size."""
+    if x.dim() != 2:
+        raise ValueError("x must be M x K")
     M, K = x.shape
     out_f32 = 1 if y.dtype == torch.float32 else 0
     if not out_f32 and y.dtype != x.dtype:
         raise ValueError("y must be float32 or x's dtype")
+    npk, nb, nsc = _storage_sizes(N * K)
+    _req(x, "x", None)
+    _req(packed, "packed", (torch.uint8,), npk)
+    _req(codes8, "codes8", (torch.uint8,), nb)
+    _req(scales, "scales", (torch.float32,), nsc)
+    _req(y, "y", None, M * N)
+    _req(workspace, "workspace", None, optional=True)
+    _req(dev_flag, "dev_flag", (torch.int32,), 1, optional=True)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(library().aqnf4_nf4_linear(_ptr(x), dtype_code(x.dtype), M, K, _ptr(packed),
                                       _ptr(codes8), _ptr(scales), N, _ptr(y), out_f32,
@@ -255,6 +326,14 @@ def aqnf4_select_blocks(sq_err: torch.Tensor, sq_w: torch.Tensor, block_of: torc
                         cost_bytes: torch.Tensor, num_blocks: int, budget_bytes: int, order: int,
                         block_rank: torch.Tensor, block_err: Optional[torch.Tensor],
                         k_out: torch.Tensor, stream=None) -> None:
+    L = sq_err.numel()
+    _req(sq_err, "sq_err", (torch.float64,))
+    _req(sq_w, "sq_w", (torch.float64,), L)
+    _req(block_of, "block_of", (torch.int32,), L)
+    _req(cost_bytes, "cost_bytes", (torch.int64,), L)
+    _req(block_rank, "block_rank", (torch.int32,), num_blocks)
+    _req(block_err, "block_err", (torch.float32,), num_blocks, optional=True)
+    _req(k_out, "k_out", (torch.int32,), 1)
     _check(library().aqnf4_select_blocks(_ptr(sq_err), _ptr(sq_w), _ptr(block_of),
                                          _ptr(cost_bytes), sq_err.numel(), num_blocks,
                                          budget_bytes, order, _ptr(block_rank), _ptr(block_err),

@@ -6,6 +6,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 import oracle
 from quantized_lora_setup_b200 import aqnf4
@@ -162,3 +163,51 @@ def test_binding_names_match_the_header():
         if name in ("aqnf4_status_string",):
             continue
         assert callable(getattr(aqnf4, name)), name
+
+
+class _FakeCuda:
+    """Stands in for a CUDA tensor in the binding's argument checks (no device needed)."""
+
+    def __init__(self, n, dtype, contiguous=True):
+        self.is_cuda, self.dtype, self._n, self._c = True, dtype, n, contiguous
+
+    def numel(self):
+        return self._n
+
+    def is_contiguous(self):
+        return self._c
+
+
+def test_binding_argument_checks():
+    req = aqnf4._req
+    req(None, "x", None, optional=True)
+    req(_FakeCuda(10, torch.uint8), "x", (torch.uint8,), 10)
+    for bad, msg in ((_FakeCuda(9, torch.uint8), "at least 10"),
+                     (_FakeCuda(10, torch.int8), "dtype"),
+                     (_FakeCuda(10, torch.uint8, contiguous=False), "contiguous"),
+                     (torch.zeros(10, dtype=torch.uint8), "CUDA")):
+        with pytest.raises(ValueError, match=msg):
+            req(bad, "x", (torch.uint8,), 10)
+    with pytest.raises(ValueError, match="required"):
+        req(None, "x", None)
+    # storage sizes of n weights: packed bytes, 64-element blocks, 256-block DQ scales
+    assert aqnf4._storage_sizes(1) == (1, 1, 1)
+    assert aqnf4._storage_sizes(16384) == (8192, 256, 1)
+    assert aqnf4._storage_sizes(16385) == (8193, 257, 2)
+
+
+def test_wrappers_reject_host_tensors_before_any_launch():
+    before = aqnf4.library().aqnf4_launch_count()
+    w = torch.zeros(128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        aqnf4.aqnf4_quantize(w, None, None)
+    with pytest.raises(ValueError, match="CUDA"):
+        aqnf4.aqnf4_dequantize(torch.zeros(64, dtype=torch.uint8), None, None,
+                               torch.zeros(2, dtype=torch.float32), 128,
+                               torch.zeros(128, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="M x K"):
+        aqnf4.aqnf4_nf4_linear(torch.zeros(64, dtype=torch.bfloat16), None, None, None, 1,
+                               torch.zeros(1, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="CUDA"):
+        aqnf4.make_layers([{"w": w}])
+    assert aqnf4.library().aqnf4_launch_count() == before
