@@ -185,8 +185,8 @@ AQNF4_API aqnf4_status aqnf4_layer_error_noalloc(const aqnf4_layer* layers, int3
    storage, and the products are summed in binary32.
    x (device, M x K, row-major, dtype, 16-byte aligned); packed (device, N*K/2 bytes,
    16-byte aligned), codes8 (device, N*K/64 bytes), scales (device, ceil(N*K/16384) floats):
-   the layer's storage as aqnf4_layer_error writes it; y (device, M x N, row-major): float
-   when out_f32 != 0, else dtype.  K must be a positive multiple of 64, so that each row of
+   the layer's storage as aqnf4_layer_error writes it; y (device, M x N, row-major,
+   16-byte aligned): float when out_f32 != 0, else dtype.  K must be a positive multiple of 64, so that each row of
    the layer is whole NF4 blocks.  workspace (optional, device, 16-byte aligned) of ws_bytes:
    when the output has too few 256 x 256 tiles to fill the GPU, K is split over several thread
    blocks whose binary32 partial sums go there and are then added in a fixed order; with at

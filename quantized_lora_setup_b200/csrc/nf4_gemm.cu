@@ -455,8 +455,9 @@ extern "C" aqnf4_status aqnf4_nf4_linear(const void* x, int32_t dtype, int64_t M
   if (M > (int64_t(1) << 31) - kBM || N > (int64_t(1) << 31) - kBN || K > (int64_t(1) << 31))
     return AQNF4_ERR_INVALID_ARG;
   if (!valid_dtype(dtype)) return AQNF4_ERR_DTYPE;
+  // y: the epilogue stores whole 16-byte vectors of a row when N allows it
   if (!is_aligned(x, 16) || !is_aligned(packed, 16) || !is_aligned(scales, 4) ||
-      !is_aligned(y, out_f32 ? 4 : 2) || !is_aligned(dev_flag, 4))
+      !is_aligned(y, 16) || !is_aligned(dev_flag, 4))
     return AQNF4_ERR_ALIGNMENT;
   const Tables* tb = default_tables();
   const EncodeTiledFn encode = encode_tiled();

@@ -113,6 +113,10 @@ def test_nf4_linear_rejects_bad_shapes():
     a = list(args)
     a[0] = V(0x1008)
     assert lib.aqnf4_nf4_linear(*a) == aqnf4.AQNF4_ERR_ALIGNMENT
+    for out_f32, y in ((1, 0x5004), (0, 0x5002)):  # y must allow 16-byte vector stores
+        a = list(args)
+        a[8], a[9] = V(y), out_f32
+        assert lib.aqnf4_nf4_linear(*a) == aqnf4.AQNF4_ERR_ALIGNMENT, (out_f32, y)
     assert lib.aqnf4_launch_count() == before
     assert aqnf4.aqnf4_nf4_linear_workspace_size(4, 8, 96) == 0
 
