@@ -211,3 +211,35 @@ def test_wrappers_reject_host_tensors_before_any_launch():
     with pytest.raises(ValueError, match="CUDA"):
         aqnf4.make_layers([{"w": w}])
     assert aqnf4.library().aqnf4_launch_count() == before
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """The header compiles as strict C11 and a C program links against the library: the
+    codebook, cost closed form and early argument checks it prints match the oracle."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    lib_dir = os.path.dirname(aqnf4.LIB)
+    exe = str(tmp_path / "abi_consumer")
+    src = os.path.join(os.path.dirname(__file__), "abi_consumer.c")
+    subprocess.run([cc, "-std=c11", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", INCLUDE,
+                    src, "-o", exe, "-L", lib_dir, "-laqnf4", f"-Wl,-rpath,{lib_dir}"],
+                   check=True)
+    out = subprocess.run([exe], check=True, capture_output=True, text=True).stdout
+    rows = [line.split() for line in out.splitlines()]
+    levels, mids = oracle.codebook()
+    got_l = [float.fromhex(r[2]) for r in rows if r[0] == "level"]
+    got_m = [float.fromhex(r[2]) for r in rows if r[0] == "mid"]
+    assert np.array_equal(np.float32(got_l), np.asarray(levels, np.float32))
+    assert np.array_equal(np.float32(got_m), np.asarray(mids, np.float32))
+    for r in rows:
+        if r[0] == "cost":
+            assert int(r[2]) == oracle.cost_bytes(int(r[1]))
+    kv = {r[0]: r[1] for r in rows if len(r) == 2}
+    assert int(kv["layer_error_null_w"]) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert int(kv["dequantize_null"]) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert int(kv["nf4_linear_bad_k"]) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert int(kv["launches"]) == 0
+    assert out.splitlines()[-1] == "status " + aqnf4.status_string(aqnf4.AQNF4_ERR_ALIGNMENT)
