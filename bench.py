@@ -808,6 +808,17 @@ def bench_e2e(args, weights, step, sel, kout, dev, stream, world, total_weight_b
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4 + 4 * L, "steps": steps}
 
 
+def fixed_duration_chunks(run_chunk, max_over_ranks, min_ms):
+    """Run chunks until their summed time reaches min_ms.  Each chunk's time is the maximum
+    over ranks (max_over_ranks is a collective), so every rank sees the same sum and stops
+    after the same number of chunks.  Returns (chunks, summed ms)."""
+    chunks, total = 0, 0.0
+    while total < min_ms:
+        total += max_over_ranks(run_chunk())
+        chunks += 1
+    return chunks, total
+
+
 def bench_protocol(step, dev, stream, world, total_weight_bytes, ms_per_step,
                    min_seconds=2.0):
     """The source pages' timing rules for the scoring step: the same step is run as two
@@ -819,22 +830,27 @@ def bench_protocol(step, dev, stream, world, total_weight_bytes, ms_per_step,
     import torch.distributed as dist
 
     chunk = max(1, int(250.0 / max(ms_per_step, 1e-3)))
+
+    def run_chunk():
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(chunk):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b)
+
+    def max_over_ranks(ms):
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
     arms = {}
     for arm in ("a", "b"):
-        total_ms, steps = 0.0, 0
-        while total_ms < min_seconds * 1e3:
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            torch.cuda.synchronize(dev)
-            a.record(stream)
-            for _ in range(chunk):
-                step()
-            b.record(stream)
-            torch.cuda.synchronize(dev)
-            ms = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
-            if world > 1:
-                dist.all_reduce(ms, op=dist.ReduceOp.MAX)
-            total_ms += float(ms.item())
-            steps += chunk
+        chunks, total_ms = fixed_duration_chunks(run_chunk, max_over_ranks, min_seconds * 1e3)
+        steps = chunks * chunk
         arms[arm] = {"steps": steps, "seconds": total_ms / 1e3,
                      "value": total_weight_bytes * steps / (total_ms / 1e3) / 1e9}
     va, vb = arms["a"]["value"], arms["b"]["value"]

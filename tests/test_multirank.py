@@ -92,3 +92,37 @@ def test_two_ranks_select_like_one(tmp_path):
         got = np.load(tmp_path / f"rank{rank}.npy")
         assert np.array_equal(got[:L], ref_scores)
         assert got[L:].astype(int).tolist() == ref_sel
+
+
+def _duration_worker(rank, world, port, result_dir):
+    """bench.py's fixed-duration loop with a per-rank chunk time (rank 1 is slower and
+    uneven): the max-over-ranks collective must make both ranks take the same chunks."""
+    import importlib.util
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(root, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    try:
+        times = iter([100.0] * 50) if rank == 0 else iter([50.0, 500.0] * 25)
+
+        def max_over_ranks(ms):
+            t = torch.tensor([ms], dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            return float(t.item())
+
+        chunks, total = bench.fixed_duration_chunks(lambda: next(times), max_over_ranks, 2000.0)
+        np.save(os.path.join(result_dir, f"dur{rank}.npy"), np.array([chunks, total]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_fixed_duration_loop_agrees_across_ranks(tmp_path):
+    port = _free_port()
+    mp.start_processes(_duration_worker, args=(2, port, str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+    got = [np.load(tmp_path / f"dur{r}.npy").tolist() for r in range(2)]
+    # per chunk max(100, 50 or 500) = 100, 500, 100, 500, ...; the running sum first
+    # reaches 2000 ms at 2400 after 8 chunks
+    assert got[0] == got[1] == [8.0, 2400.0]
