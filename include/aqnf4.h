@@ -3,16 +3,18 @@
  *
  * The pass quantizes each linear layer of a model to 4-bit NormalFloat (NF4) in blocks of
  * 64 elements, double-quantizes the per-block absmax constants to 8 bits in blocks of 256,
- * measures each layer's relative reconstruction error, and keeps the top-K layers in 16 bits
- * under a byte budget.  A standalone NF4 -> 16-bit dequantization comes with it.
+ * measures each layer's relative reconstruction error, and picks the K largest-error layers
+ * to stay in 16 bits within a byte budget.  A standalone NF4 -> 16-bit dequantization comes with it.
  *
  * Sources (page title, section):
  *   "QLoRA" (ai360xpert.com), "How It Works": NF4 spreads the weights evenly over its 16
- *       values; double quantization quantizes the quantization constants (about 0.37 bits
- *       per parameter saved); weights are dequantized to 16 bits on the fly.
+ *       values; the per-block scales get an 8-bit encoding of their own, worth about 0.37
+ *       bits per weight; training turns the 4-bit weights back into 16-bit values whenever
+ *       a pass needs them.
  *   "QLoRA Explained" (devtoolshub.net), "NF4", "Double Quantization".
- *   arxivdaily 2608.23816, "English abstract": one pass over the weights ranks layers by
- *       NF4 reconstruction error and keeps the top-K in fp16 under a memory budget.
+ *   arxivdaily 2608.23816, "English abstract": a single sweep over the weights orders the
+ *       layers by their NF4 error and holds the highest-error ones in 16 bits, as many as a
+ *       byte budget allows.
  *   "AQLoRA: A Zero-Search Recipe for Fast Quantized LoRA Fine-Tuning", "Technical Details":
  *       every layer is ranked; the memory budget is configurable.
  *
@@ -70,7 +72,7 @@ typedef enum { AQNF4_F16 = 0, AQNF4_BF16 = 1 } aqnf4_dtype;
 /* aqnf4_layer.flags bits. */
 enum {
   /* Score the layer as NF4 + double quantization stores it ("QLoRA", "How It Works": the
-     quantization constants are quantized in turn): w_hat is rebuilt from the DQ constant
+     block scales are themselves stored at 8 bits): w_hat is rebuilt from the DQ constant
      a'_b = fl(fl(code8_b / 255) * s) of its block, exactly what aqnf4_dequantize returns
      from packed + codes8 + scales, instead of the binary32 absmax a_b.  The codes, packed
      bytes, absmax, codes8 and scales written are the same either way. */
@@ -120,8 +122,8 @@ AQNF4_API aqnf4_status aqnf4_codebook(double p_max, float levels[16], float mids
 AQNF4_API aqnf4_status aqnf4_quantize(const void* w, int32_t dtype, int64_t n, uint8_t* packed,
                             float* absmax, int32_t* dev_flag, cudaStream_t stream);
 
-/* Double quantization of an absmax array ("QLoRA", "How It Works": quantizing the
-   quantization constants; "QLoRA Explained", "Double Quantization").
+/* Double quantization of an absmax array ("QLoRA", "How It Works": the block scales get
+   an 8-bit encoding of their own; "QLoRA Explained", "Double Quantization").
    absmax (device, 4-byte aligned): nb constants.  For each block of 256 constants
    s = max a (NaN if any is NaN) is stored in scales[d] and each constant becomes
    code8 = round_half_even(fl(fl(a / s) * 255)); s = 0 gives codes 0; a NaN or infinite s
@@ -132,7 +134,8 @@ AQNF4_API aqnf4_status aqnf4_quantize(const void* w, int32_t dtype, int64_t n, u
 AQNF4_API aqnf4_status aqnf4_double_quant(const float* absmax, int64_t nb, uint8_t* codes8,
                                 float* scales, int32_t* dev_flag, cudaStream_t stream);
 
-/* NF4 -> 16-bit dequantization ("QLoRA", "How It Works": dequantized to 16 bits on the fly).
+/* NF4 -> 16-bit dequantization ("QLoRA", "How It Works": the 16-bit values training computes
+   with are rebuilt from the 4-bit storage when needed).
    packed (device, 16-byte aligned): ceil(n/2) bytes.  The block constant is
    a' = fl(fl(code8/255) * scales[b/256]) when codes8 is non-NULL (then scales is required),
    else a' = absmax[b].  out[i] = dtype_rn(fl(levels[code_i] * a')).
@@ -178,8 +181,8 @@ AQNF4_API aqnf4_status aqnf4_layer_error_noalloc(const aqnf4_layer* layers, int3
                                                  double* sq_err, double* sq_w, float* rel_err,
                                                  int32_t* dev_flag, cudaStream_t stream);
 
-/* Forward product of a layer stored in NF4 + DQ ("QLoRA", "How It Works": the 4-bit weights
-   are dequantized to 16 bits on the fly for the forward pass), on the tensor cores with the
+/* Forward product of a layer stored in NF4 + DQ ("QLoRA", "How It Works": a training pass
+   works on 16-bit values rebuilt from the 4-bit storage), on the tensor cores with the
    dequantization fused in: y = x w_hat^T, where w_hat (N x K) is exactly what
    aqnf4_dequantize(packed, codes8, scales, NULL, N*K, dtype, ...) returns for the layer's
    storage, and the products are summed in binary32.
@@ -205,8 +208,9 @@ AQNF4_API aqnf4_status aqnf4_nf4_linear(const void* x, int32_t dtype, int64_t M,
    it does not split).  Host only. */
 AQNF4_API size_t aqnf4_nf4_linear_workspace_size(int64_t M, int64_t N, int64_t K);
 
-/* Top-K under a byte budget (arxivdaily 2608.23816, "English abstract": keep the top-K in
-   fp16 under a memory budget; "AQLoRA: ...", "Technical Details": configurable budget).
+/* Top-K under a byte budget (arxivdaily 2608.23816, "English abstract": the highest-error
+   layers stay in 16 bits while a byte budget allows; "AQLoRA: ...", "Technical Details":
+   the budget is a setting).
    Layers are ranked by rel_err descending, equal scores by lower index first, NaN scores
    last.  Walking the ranking, layers are kept until the next one would exceed k_cap layers
    (k_cap < 0: no cap) or push the summed cost_bytes above budget_bytes.

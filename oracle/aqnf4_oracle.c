@@ -16,18 +16,19 @@
  *
  * Sources (page title, section):
  *   [QLoRA/HIW]  "QLoRA" (ai360xpert.com), "How It Works": NF4 gives each of its 16
- *                values an equal share of the weights; double quantization quantizes
- *                the quantization constants and saves about 0.37 bits per parameter;
- *                weights are dequantized to 16 bits on the fly.
+ *                values an equal share of the weights; the per-block scales get an
+ *                8-bit encoding of their own, worth about 0.37 bits per weight; a
+ *                training pass computes with 16-bit values rebuilt from the storage.
  *   [QLoRA/Idea] "QLoRA" (ai360xpert.com), "The Idea": NF4 is built for normally
  *                distributed weights.
  *   [QLE/NF4]    "QLoRA Explained" (devtoolshub.net), "NF4" and "4-Bit Quantization in
  *                QLoRA": the data type follows the normal distribution of weights.
- *   [QLE/DQ]     "QLoRA Explained", "Double Quantization": constants map compressed
- *                values back to their numerical range; DQ quantizes those constants.
- *   [AQLoRA/abs] arxivdaily 2608.23816, "English abstract": one pass over the weights
- *                ranks layers by NF4 reconstruction error and keeps the top-K in fp16
- *                under a memory budget; the quality setting costs 0.2 GiB more memory.
+ *   [QLE/DQ]     "QLoRA Explained", "Double Quantization": the per-block
+ *                constants restore each block's range, and DQ stores them compressed too.
+ *   [AQLoRA/abs] arxivdaily 2608.23816, "English abstract": a single sweep over the
+ *                weights orders the layers by their NF4 error and holds the highest-error
+ *                ones in 16 bits while a byte budget allows; the quality setting needs
+ *                0.2 GiB of extra memory.
  *   [AQLoRA/TD]  "AQLoRA: A Zero-Search Recipe for Fast Quantized LoRA Fine-Tuning",
  *                "Technical Details": every layer is ranked; the budget is configurable.
  *
@@ -384,7 +385,7 @@ int oracle_layer_error_dq(const uint16_t* w, int dtype, int64_t n, const float l
 
 /* ------------------------------------------------------------- dequantize */
 
-/* NF4 -> 16-bit ([QLoRA/HIW]: dequantized to 16 bits on the fly).
+/* NF4 -> 16-bit ([QLoRA/HIW]: the 16-bit values a training pass computes with).
    With codes8 != NULL the block constant is a' = fl(fl(code8/255) * scale[b/256]);
    otherwise a' = absmax[b].  out: n 16-bit values of out_dtype. */
 void oracle_dequantize(const uint8_t* packed, const uint8_t* codes8, const float* scales,
@@ -408,8 +409,8 @@ void oracle_dequantize(const uint8_t* packed, const uint8_t* codes8, const float
 
 /* ------------------------------------------------ linear layer on NF4 weights */
 
-/* The forward product of a layer kept in NF4 + DQ ([QLoRA/HIW]: the 4-bit weights are
-   dequantized to 16 bits on the fly for the forward pass): y = x w_hat^T with
+/* The forward product of a layer kept in NF4 + DQ ([QLoRA/HIW]: a training pass computes
+   with 16-bit values rebuilt from the 4-bit storage): y = x w_hat^T with
    x: M x K 16-bit (x_dtype), row-major; w_hat: the N x K layer rebuilt in w_dtype from its
    packed codes, codes8 and scales exactly as oracle_dequantize does; y: M x N in binary64
    (every product and sum exact up to binary64 rounding).  yabs (optional) receives

@@ -1,7 +1,7 @@
 // dequant.cu -- NF4 -> 16-bit dequantization (aqnf4_dequantize).
 //
-// "QLoRA", "How It Works": the 4-bit weights are dequantized to 16 bits on the fly for the
-// forward and backward pass.  For element i of block b = i / 64:
+// "QLoRA", "How It Works": training computes with 16-bit values rebuilt from the 4-bit
+// storage each time a pass needs them.  For element i of block b = i / 64:
 //   a' = fl(fl(code8[b] / 255) * scales[b / 256])   (double-quantized constants), or
 //   a' = absmax[b]                                  (plain constants);
 //   out[i] = dtype_rn(fl(level[code_i] * a')).

@@ -1,7 +1,7 @@
 // double_quant.cu -- standalone double quantization of an absmax array (aqnf4_double_quant).
 //
-// "QLoRA", "How It Works": the quantization constants are themselves quantized, which saves
-// about 0.37 bits per parameter; "QLoRA Explained", "Double Quantization".  Each block of
+// "QLoRA", "How It Works": the per-block scales get an 8-bit encoding of their own, worth
+// about 0.37 bits per weight; "QLoRA Explained", "Double Quantization".  Each block of
 // 256 constants keeps one binary32 scale s = max a and one byte per constant,
 // code8 = round_half_even(fl(fl(a / s) * 255)).  The fused pass in quant_score.cu applies
 // the same dq_code to the same constants, so both give identical bytes.

@@ -1,8 +1,8 @@
 // nf4_gemm.cu -- the forward product of a layer stored in NF4 + DQ on the tensor cores
 // (aqnf4_nf4_linear): y = x w_hat^T.
 //
-// "QLoRA", "How It Works": the 4-bit weights are dequantized to 16 bits on the fly for the
-// forward and backward pass.  Here that dequantization happens inside the GEMM: w_hat never
+// "QLoRA", "How It Works": a training pass computes with 16-bit values rebuilt from the
+// 4-bit storage.  Here that rebuilding happens inside the GEMM: w_hat never
 // exists in HBM.  For element (n, k) of the N x K layer (block b = (n K + k) / 64):
 //   a'_b = fl(fl(code8_b / 255) * scales[b / 256]),  w_hat = dtype_rn(fl(level[code] * a'_b)),
 // bit for bit what aqnf4_dequantize writes; then y = x w_hat^T with binary32 accumulation.

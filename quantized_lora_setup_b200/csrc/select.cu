@@ -1,9 +1,9 @@
 // select.cu -- top-K layers under a byte budget (aqnf4_select_topk) and the block-level
 // selection of the speed setting (aqnf4_select_blocks).
 //
-// arxivdaily 2608.23816, "English abstract": the pass ranks layers by NF4 reconstruction
-// error and keeps the top-K in fp16 under a memory budget; "AQLoRA: A Zero-Search Recipe
-// for Fast Quantized LoRA Fine-Tuning", "Technical Details": the budget is configurable.
+// arxivdaily 2608.23816, "English abstract": the layers are ordered by their NF4 error and
+// the highest-error ones stay in 16 bits while a byte budget allows; "AQLoRA: A Zero-Search
+// Recipe for Fast Quantized LoRA Fine-Tuning", "Technical Details": the budget is a setting.
 //
 // Ranking: score descending, equal scores by lower layer index, NaN scores last.  A model
 // has a few hundred layers, so one CTA of 1024 threads computes every layer's rank by

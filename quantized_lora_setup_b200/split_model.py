@@ -1,9 +1,10 @@
 """The split model the selection describes: top-K layers in 16 bits, the rest in NF4 + DQ.
 
-arxivdaily 2608.23816, "English abstract": one pass over the weights ranks the layers by NF4
-reconstruction error and keeps the top-K in fp16 under a memory budget; those layers skip
-dequantization.  "QLoRA", "How It Works": the other layers are stored as 4-bit NF4 with
-double-quantized constants and dequantized to 16 bits on the fly.
+arxivdaily 2608.23816, "English abstract": a single sweep over the weights orders the layers
+by their NF4 error, and the highest-error ones stay in 16 bits while a byte budget allows, so
+training never has to rebuild them.  "QLoRA", "How It Works": every other layer is held as
+4-bit NF4 with 8-bit-encoded block scales, and its 16-bit values are rebuilt whenever a pass
+needs them.
 
 :func:`materialize` runs the fused pass over every layer (which writes each layer's NF4 + DQ
 storage while it scores it), selects on the device, then keeps per layer exactly one copy:
