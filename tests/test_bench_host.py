@@ -31,3 +31,26 @@ def test_dequant_alg_bytes(bench):
     assert bench.dequant_alg_bytes(n) == n // 2 + nb + 4 * ((nb + 255) // 256) + 2 * n
     # a ragged tail: 100 elements = 2 blocks, 1 scale
     assert bench.dequant_alg_bytes(100) == 50 + 2 + 4 + 200
+
+
+def _profile_commands():
+    """Every `python bench.py ...` command line the profile summaries give (backslash
+    continuations joined, inline-code backticks and trailing prose dropped)."""
+    import glob
+    import re
+    cmds = []
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        text = open(path).read().replace("\\\n", " ")
+        for line in text.splitlines():
+            for m in re.finditer(r"python bench\.py((?:\s+--?[\w-]+(?:[ =](?!--)[^\s`]+)?)*)", line):
+                cmds.append((os.path.basename(path), m.group(1).split()))
+    return cmds
+
+
+def test_profile_commands_parse(bench, monkeypatch):
+    """The commands the profiles record still parse with bench.py's own arguments."""
+    cmds = _profile_commands()
+    assert len(cmds) >= 5
+    for name, argv in cmds:
+        monkeypatch.setattr("sys.argv", ["bench.py"] + argv)
+        bench.parse_args()  # exits on an unknown or malformed argument
