@@ -152,7 +152,7 @@ def run_reference(args):
         oracle_pass(sample)
     dt = time.perf_counter() - t0
     value = 2 * elems * args.steps / dt / 1e9
-    desc = (f"{len(sample)} slices of up to {per_thread} elements (the first elements of the "
+    desc = (f"{len(sample)} slices of {sample[0][0].size} elements (the first elements of the "
             f"first {len(sample)} layers), {elems} weights per step, one thread per slice")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
@@ -420,7 +420,7 @@ def run_native(args):
         dt = time.perf_counter() - t0
         result["cpu_baseline"] = {
             "value": 2 * elems / dt / 1e9, "unit": UNIT, "cores": len(sample), "kind": "oracle",
-            "sample": f"{len(sample)} slices of up to {per_thread} elements from the first "
+            "sample": f"{len(sample)} slices of {sample[0][0].size} elements from the first "
                       f"{len(sample)} layers ({elems} weights), quantize + DQ + error, one "
                       f"thread per slice"}
         if args.protocol:  # the pages' second oracle timing: one slice on one thread
