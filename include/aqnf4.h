@@ -19,7 +19,10 @@
  *       every layer is ranked; the memory budget is configurable.
  *
  * Conventions for every call:
- *   - The caller owns every buffer.  The library allocates nothing and frees nothing.
+ *   - The caller owns every buffer.  The library allocates nothing and frees nothing; the one
+     exception is the fixed scratch array that aqnf4_layer_error_noalloc uses (8 MiB of
+     static device memory per device, with its address cached per device after the first
+     call; the cache is not refreshed after cudaDeviceReset).
  *   - Pointers named "device" must be CUDA device (or managed) memory of the current device.
  *   - Calls with a stream argument are asynchronous on that stream (0 = legacy default
  *     stream).  The returned status covers the synchronous argument checks and the launch;
@@ -195,9 +198,11 @@ AQNF4_API aqnf4_status aqnf4_layer_error_noalloc(const aqnf4_layer* layers, int3
    blocks whose binary32 partial sums go there and are then added in a fixed order; with at
    least aqnf4_nf4_linear_workspace_size(M, N, K) bytes the split is used, otherwise the call
    runs unsplit (still correct).  dev_flag (optional, device int32) receives
-   AQNF4_ERR_TIMEOUT if a bounded wait inside the kernel gave up (y is then not written).
+   AQNF4_ERR_TIMEOUT if a bounded wait inside the kernel gave up; y is then not written by
+   the split-K sum and its tiles are not meaningful (without a dev_flag a timeout goes
+   unreported and y is undefined).
    Errors: INVALID_ARG (NULL pointer, M < 1, N < 1, K not a positive multiple of 64, sizes
-   above 2^31), DTYPE, ALIGNMENT, CUDA. */
+   above 2^31, M above 65535 * 256 = 16776960 rows), DTYPE, ALIGNMENT, CUDA. */
 AQNF4_API aqnf4_status aqnf4_nf4_linear(const void* x, int32_t dtype, int64_t M, int64_t K,
                                         const uint8_t* packed, const uint8_t* codes8,
                                         const float* scales, int64_t N, void* y,
@@ -230,6 +235,17 @@ AQNF4_API aqnf4_status aqnf4_select_topk(const float* rel_err, const int64_t* co
    normally, leaving the context usable.  Errors: INVALID_ARG, ALIGNMENT, CUDA. */
 AQNF4_API aqnf4_status aqnf4_selftest_wait_timeout(int64_t timeout_ns, int32_t* dev_flag,
                                                    int64_t* waited_ns, cudaStream_t stream);
+
+/* Diagnostic (no counterpart on the pages).  The fused pass takes fl(1/a) and fl(a/s) with a
+   short Newton-Raphson form (the hardware reciprocal approximation and one fused
+   multiply-add correction) that is exact for the 16-bit values it meets.  This call
+   evaluates, for each i < n, out[4i] = that reciprocal of a[i], out[4i+1] = CUDA's
+   correctly rounded __frcp_rn(a[i]), out[4i+2] = the short quotient a[i] / s[i] and
+   out[4i+3] = CUDA's __fdiv_rn(a[i], s[i]), so a test can compare them.  a, s (device
+   float[n]) are inputs, out (device float[4n], 16-byte aligned) the output.
+   Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+AQNF4_API aqnf4_status aqnf4_selftest_division(const float* a, const float* s, int64_t n,
+                                               float* out, cudaStream_t stream);
 
 /* Incremental bytes of keeping an n-element layer in 16 bits instead of its NF4 storage
    (packed + codes8 + scales): 2n - (ceil(n/2) + ceil(n/64) + 4*ceil(ceil(n/64)/256)).

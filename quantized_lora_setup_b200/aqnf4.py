@@ -94,6 +94,8 @@ def library() -> ctypes.CDLL:
     lib.aqnf4_select_topk.restype = st
     lib.aqnf4_selftest_wait_timeout.argtypes = [i64, P, P, P]
     lib.aqnf4_selftest_wait_timeout.restype = st
+    lib.aqnf4_selftest_division.argtypes = [P, P, i64, P, P]
+    lib.aqnf4_selftest_division.restype = st
     lib.aqnf4_nf4_linear.argtypes = [P, i32, i64, i64, P, P, P, i64, P, i32, P,
                                      ctypes.c_size_t, P, P]
     lib.aqnf4_nf4_linear.restype = st
@@ -289,6 +291,18 @@ def aqnf4_selftest_wait_timeout(timeout_ns: int, dev_flag: torch.Tensor,
                                 waited_ns: Optional[torch.Tensor] = None, stream=None) -> None:
     _check(library().aqnf4_selftest_wait_timeout(int(timeout_ns), _ptr(dev_flag), _ptr(waited_ns),
                                                  _stream(stream)), "aqnf4_selftest_wait_timeout")
+
+
+def aqnf4_selftest_division(a: torch.Tensor, s: torch.Tensor, out: torch.Tensor,
+                            stream=None) -> None:
+    """out[i] = (short reciprocal of a[i], __frcp_rn(a[i]), short quotient a[i]/s[i],
+    __fdiv_rn(a[i], s[i])); out is float32 (n, 4)."""
+    n = a.numel()
+    _req(a, "a", (torch.float32,))
+    _req(s, "s", (torch.float32,), n)
+    _req(out, "out", (torch.float32,), 4 * n)
+    _check(library().aqnf4_selftest_division(_ptr(a), _ptr(s), n, _ptr(out), _stream(stream)),
+           "aqnf4_selftest_division")
 
 
 def aqnf4_nf4_linear(x: torch.Tensor, packed: torch.Tensor, codes8: torch.Tensor,

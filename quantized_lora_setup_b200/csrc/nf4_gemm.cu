@@ -364,11 +364,14 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
 }
 
 // Split K: y = sum over z of the binary32 partials ws[z], added in split order (the result
-// does not depend on scheduling), converted to y's format.
+// does not depend on scheduling), converted to y's format.  If the GEMM reported a timeout in
+// the caller's flag word, some partials were never written: y is left alone.
 template <int DT>
 __global__ void __launch_bounds__(256) k_splitk_reduce(const float* __restrict__ ws, int splits,
-                                                       int64_t mn, void* y, int out_f32) {
+                                                       int64_t mn, void* y, int out_f32,
+                                                       const int32_t* flag) {
   using F = Fmt<DT>;
+  if (flag && *reinterpret_cast<const volatile int32_t*>(flag) == AQNF4_ERR_TIMEOUT) return;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < mn;
        i += static_cast<int64_t>(gridDim.x) * 256) {
     float acc = __ldcs(ws + i);
@@ -428,7 +431,7 @@ cudaError_t launch_gemm(const CUtensorMap& map, const GParams& p, cudaStream_t s
     const int64_t cap = static_cast<int64_t>(current_sm_count() > 0 ? current_sm_count() : 148) * 8;
     if (blocks > cap) blocks = cap;
     k_splitk_reduce<DT><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p.ws, p.splits, mn,
-                                                                           p.y, p.out_f32);
+                                                                           p.y, p.out_f32, p.flag);
     count_launches(1);
   }
   return cudaGetLastError();
@@ -454,6 +457,7 @@ extern "C" aqnf4_status aqnf4_nf4_linear(const void* x, int32_t dtype, int64_t M
     return AQNF4_ERR_INVALID_ARG;
   if (M > (int64_t(1) << 31) - kBM || N > (int64_t(1) << 31) - kBN || K > (int64_t(1) << 31))
     return AQNF4_ERR_INVALID_ARG;
+  if ((M + kBM - 1) / kBM > 65535) return AQNF4_ERR_INVALID_ARG;  // row tiles go on grid y
   if (!valid_dtype(dtype)) return AQNF4_ERR_DTYPE;
   // y: the epilogue stores whole 16-byte vectors of a row when N allows it
   if (!is_aligned(x, 16) || !is_aligned(packed, 16) || !is_aligned(scales, 4) ||

@@ -17,7 +17,7 @@
 // Work decomposition (B200): a tile is 16384 consecutive elements of one layer (one DQ
 // block, 256 NF4 blocks).  A persistent CTA of 128 threads walks tiles with a grid stride;
 // thread t owns NF4 blocks t and t + 128.  A 1-D bulk copy (TMA engine) brings each 32 KB
-// tile into shared memory; four CTAs share an SM, so one CTA's copy overlaps the others'
+// tile into shared memory; five CTAs share an SM, so one CTA's copy overlaps the others'
 // arithmetic.  Each thread reads its blocks twice with conflict-free 16-byte loads (chunk
 // order rotated per thread): once for the absmax (packed bf16x2/f16x2 max), once to code,
 // the two blocks' work interleaved.  A code does not count midpoints: an odd cubic
@@ -28,8 +28,11 @@
 // for every normalised v are built on the host (codebook.cpp).  Arithmetic on pairs uses
 // Blackwell's packed f32x2 instructions, and w_hat - x comes from the packed 16-bit w_hat
 // with one mixed-precision subtract.  Packed codes are staged in shared memory and leave with
-// coalesced 16-byte stores.  The per-tile extra work (the next bulk copy, the binary64
-// reduction) rotates over the warps so no warp is always last at a barrier.
+// coalesced 16-byte stores.  fl(1/a) and the DQ quotient fl(a/s) come from a one-step
+// Newton-Raphson form on the fused multiply-add (rcp16_rn, quot16_rn), exact for the 16-bit
+// values met here, instead of a full divide per block.  The per-tile extra work (the next
+// bulk copy, the binary64 reduction) rotates over the warps so no warp is always last at a
+// barrier.
 #include <cfloat>
 #include <mutex>
 
@@ -267,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       a[b] = F::abs_lo(m0);
       // 2^-40 <= a <= 2^40: (w_hat - x)^2 and x^2 cannot overflow or flush in binary32
       fast[b] = (a[b] >= 0x1p-40f) && (a[b] <= 0x1p40f);
-      r[b] = fast[b] ? __frcp_rn(a[b]) : 0.0f;
+      r[b] = fast[b] ? rcp16_rn(a[b]) : 0.0f;
     }
 
     // ---- the constant w_hat is rebuilt from: a, or for a DQ score the double-quantized
@@ -395,13 +398,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     for (int w = 0; w < kWarps; ++w) sdq_bits = max(sdq_bits, __float_as_uint(wmax[w]));
     const float sdq = __uint_as_float(sdq_bits);
     const int64_t blk0 = g.tin * kDqBlock;
+    // the short exact quotient needs the scale in [2^-40, 2^40]; otherwise (zero, subnormal,
+    // huge or non-finite scale) the plain correctly rounded divide
+    const bool sfast = sdq >= 0x1p-40f && sdq <= 0x1p40f;
+    const float ys = sfast ? rcp16_rn(sdq) : 0.0f;
 #pragma unroll
     for (int b = 0; b < kBpt; ++b) {
       const int blk = t + b * kThreads;
       if (blk < nblk) {
         if (L.absmax) __stcs(L.absmax + blk0 + blk, a[b]);
         if (L.codes8) __stcs(reinterpret_cast<char*>(L.codes8) + blk0 + blk,
-                             static_cast<char>(dq_code(a[b], sdq)));
+                             static_cast<char>(sfast ? dq_code_fast(a[b], sdq, ys)
+                                                     : dq_code(a[b], sdq)));
       }
     }
     if (t == 0 && L.codes8) {

@@ -1,7 +1,8 @@
-// selftest.cu -- aqnf4_selftest_wait_timeout: exercises the bounded mbarrier wait that every
-// bulk-copy consumer in this library uses, on a barrier that nothing ever completes, so the
-// give-up path (status AQNF4_ERR_TIMEOUT, kernel returns, context stays usable) can be tested
-// without a fault or a hang.
+// selftest.cu -- diagnostics.  aqnf4_selftest_wait_timeout exercises the bounded mbarrier
+// wait that every bulk-copy consumer in this library uses, on a barrier that nothing ever
+// completes, so the give-up path (status AQNF4_ERR_TIMEOUT, kernel returns, context stays
+// usable) can be tested without a fault or a hang.  aqnf4_selftest_division evaluates the
+// fused pass's short reciprocal and quotient beside CUDA's correctly rounded ones.
 #include "device.cuh"
 
 namespace aqnf4 {
@@ -22,6 +23,19 @@ __global__ void k_selftest_wait(uint64_t timeout_ns, int32_t* flag, int64_t* wai
   }
 }
 
+__global__ void k_selftest_division(const float* a, const float* s, int64_t n, float* out) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float ai = a[i], si = s[i];
+    float4 o;
+    o.x = rcp16_rn(ai);
+    o.y = __frcp_rn(ai);
+    o.z = quot16_rn(ai, si, rcp16_rn(si));
+    o.w = __fdiv_rn(ai, si);
+    reinterpret_cast<float4*>(out)[i] = o;
+  }
+}
+
 }  // namespace
 }  // namespace aqnf4
 
@@ -32,6 +46,17 @@ extern "C" aqnf4_status aqnf4_selftest_wait_timeout(int64_t timeout_ns, int32_t*
   if (timeout_ns < 1 || timeout_ns > 2000000000ll || !dev_flag) return AQNF4_ERR_INVALID_ARG;
   if (!is_aligned(dev_flag, 4) || !is_aligned(waited_ns, 8)) return AQNF4_ERR_ALIGNMENT;
   k_selftest_wait<<<1, 32, 0, stream>>>(static_cast<uint64_t>(timeout_ns), dev_flag, waited_ns);
+  count_launches(1);
+  return cudaGetLastError() == cudaSuccess ? AQNF4_OK : AQNF4_ERR_CUDA;
+}
+
+extern "C" aqnf4_status aqnf4_selftest_division(const float* a, const float* s, int64_t n,
+                                                float* out, cudaStream_t stream) {
+  if (!a || !s || !out || n < 1) return AQNF4_ERR_INVALID_ARG;
+  if (!is_aligned(a, 4) || !is_aligned(s, 4) || !is_aligned(out, 16)) return AQNF4_ERR_ALIGNMENT;
+  const int64_t blocks = (n + 255) / 256;
+  k_selftest_division<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), 256, 0, stream>>>(
+      a, s, n, out);
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? AQNF4_OK : AQNF4_ERR_CUDA;
 }

@@ -149,6 +149,16 @@ def test_argument_checks_return_before_any_launch(lib):
     assert lib.aqnf4_selftest_wait_timeout(3_000_000_000, V(0x100), None, None) == aqnf4.AQNF4_ERR_INVALID_ARG
     assert lib.aqnf4_selftest_wait_timeout(1000, None, None, None) == aqnf4.AQNF4_ERR_INVALID_ARG
     assert lib.aqnf4_selftest_wait_timeout(1000, V(0x102), None, None) == aqnf4.AQNF4_ERR_ALIGNMENT
+    # fused GEMM: row tiles beyond the grid's y limit are rejected up front
+    gemm = [V(0x100), aqnf4.AQNF4_BF16, 65535 * 256, 64, V(0x200), V(0x300), V(0x400), 256,
+            V(0x500), 0, None, 0, None, None]
+    big = list(gemm)
+    big[2] = 65535 * 256 + 1
+    assert lib.aqnf4_nf4_linear(*big) == aqnf4.AQNF4_ERR_INVALID_ARG
+    # division diagnostic
+    assert lib.aqnf4_selftest_division(V(0x100), V(0x200), 0, V(0x300), None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert lib.aqnf4_selftest_division(None, V(0x200), 4, V(0x300), None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert lib.aqnf4_selftest_division(V(0x100), V(0x200), 4, V(0x308), None) == aqnf4.AQNF4_ERR_ALIGNMENT
     assert lib.aqnf4_launch_count() == before
 
 
