@@ -2,12 +2,19 @@
 
 Every layer of the 1.4B-, 7B- and 14B-shaped models goes through one aqnf4_layer_error
 call (fused quantize + pack + double quantization + error), exactly as in bench.py.  The
-oracle then recomputes a sample of layers one by one (first, middle, last, and one of
-each value distribution): packed codes, DQ bytes and scales must be bit-exact and the
-scores within 1e-5.  The selection at every budget must equal the oracle's selection on
-the same score vector.  The standalone dequantization of a 28672x8192 matrix is checked
-on DQ-block-aligned slices, and one layer of more than 2^32 elements on sampled tiles.
+oracle then scores EVERY layer on the host cores: each layer's sums and relative error must
+agree within 1e-5, and at every budget the GPU's kept set must equal the oracle's selection
+on the oracle's own scores (arxivdaily 2608.23816, "English abstract": the layers are
+ranked by NF4 error and the top ones kept under a byte budget).  Where the GPU's scores at
+the cut lie within 2e-5 of each other the two sets may differ legitimately; such a budget
+is reported as tie-ambiguous (a warning) instead of failing.  On a sample of layers (first,
+middle, last, one of each value distribution) the oracle also rebuilds the storage: packed
+codes, DQ bytes and scales bit-exact.  The
+standalone dequantization of a 28672x8192 matrix is checked on DQ-block-aligned slices,
+and one layer of more than 2^32 elements on sampled tiles.
 """
+import os
+import warnings
 from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
@@ -42,8 +49,28 @@ def _oracle_layer(args):
     return op, oc, osc, ose, osw, orel
 
 
+def _oracle_score(args):
+    w_dev, dt = args
+    return oracle.layer_error(synth.bits_u16(w_dev.cpu()), dt)
+
+
+def _selection_status(gpu_rel, ora_rel, cost, budget, k_cap, gpu_sel):
+    """'exact' when the GPU kept set equals the oracle's selection on the oracle's scores;
+    'tie-ambiguous' when it does not but the GPU scores at the cut are within 2e-5 of each
+    other; 'mismatch' otherwise."""
+    if sorted(gpu_sel) == sorted(oracle.select_topk(ora_rel, cost, budget, k_cap)):
+        return "exact"
+    order = oracle.select_topk(gpu_rel, cost, 1 << 62, -1)
+    k = len(gpu_sel)
+    if 0 < k < len(order):
+        a, b = gpu_rel[order[k - 1]], gpu_rel[order[k]]
+        if abs(a - b) <= 2e-5 * max(abs(a), abs(b)):
+            return "tie-ambiguous"
+    return "mismatch"
+
+
 @pytest.mark.parametrize("name", ["1.4b", "7b", "14b"])
-def test_full_model_sampled_layers(cuda, name):
+def test_full_model_every_layer_and_selection(cuda, name):
     wl = synth.workload(name)
     weights = [synth.layer_device(s, wl.seed, i, cuda) for i, s in enumerate(wl.layers)]
     stor = [aqnf4.NF4Storage(w.numel(), cuda) for w in weights]
@@ -53,18 +80,16 @@ def test_full_model_sampled_layers(cuda, name):
     se_h, sw_h = se.cpu().numpy(), sw.cpu().numpy()
     assert np.all(np.isfinite(rel_h)) and np.all(rel_h > 0)
 
-    sample = _sample(wl)
-    jobs = [(weights[i].cpu(), DT[wl.layers[i].dtype]) for i in sample]
-    with ThreadPoolExecutor(max_workers=len(jobs)) as ex:
-        results = list(ex.map(_oracle_layer, jobs))
-    for i, (op, oc, osc, ose, osw, orel) in zip(sample, results):
-        assert np.array_equal(stor[i].packed.cpu().numpy(), op), f"packed, layer {i}"
-        assert np.array_equal(stor[i].codes8.cpu().numpy(), oc), f"codes8, layer {i}"
-        assert np.array_equal(stor[i].scales.cpu().numpy().view(np.uint32),
-                              osc.view(np.uint32)), f"scales, layer {i}"
-        assert se_h[i] == pytest.approx(ose, rel=RTOL)
-        assert sw_h[i] == pytest.approx(osw, rel=RTOL)
-        assert rel_h[i] == pytest.approx(orel, rel=RTOL)
+    # the oracle scores every layer, one layer per host thread at a time
+    jobs = [(w, DT[s.dtype]) for w, s in zip(weights, wl.layers)]
+    with ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as ex:
+        scores = list(ex.map(_oracle_score, jobs))
+    ose = np.array([x[0] for x in scores])
+    osw = np.array([x[1] for x in scores])
+    orel = np.array([x[2] for x in scores], np.float32)
+    np.testing.assert_allclose(se_h, ose, rtol=RTOL)
+    np.testing.assert_allclose(sw_h, osw, rtol=RTOL)
+    np.testing.assert_allclose(rel_h, orel, rtol=RTOL)
 
     cost = np.array([aqnf4.aqnf4_cost_bytes(s.numel) for s in wl.layers], np.int64)
     cost_d = torch.from_numpy(cost).to(cuda)
@@ -73,6 +98,21 @@ def test_full_model_sampled_layers(cuda, name):
         got = sel.cpu().numpy()[: k.item()].tolist()
         assert got == oracle.select_topk(rel_h, cost, budget, wl.k_cap)
         assert sum(cost[got]) <= budget
+        status = _selection_status(rel_h, orel, cost, budget, wl.k_cap, got)
+        assert status != "mismatch", (name, budget)
+        if status == "tie-ambiguous":
+            warnings.warn(f"{name}, budget {budget}: kept set tie-ambiguous at the cut")
+
+    # the storage of sampled layers, bit for bit
+    sample = _sample(wl)
+    jobs = [(weights[i].cpu(), DT[wl.layers[i].dtype]) for i in sample]
+    with ThreadPoolExecutor(max_workers=len(jobs)) as ex:
+        results = list(ex.map(_oracle_layer, jobs))
+    for i, (op, oc, osc, _, _, _) in zip(sample, results):
+        assert np.array_equal(stor[i].packed.cpu().numpy(), op), f"packed, layer {i}"
+        assert np.array_equal(stor[i].codes8.cpu().numpy(), oc), f"codes8, layer {i}"
+        assert np.array_equal(stor[i].scales.cpu().numpy().view(np.uint32),
+                              osc.view(np.uint32)), f"scales, layer {i}"
 
 
 def test_full_size_dequantize(cuda):

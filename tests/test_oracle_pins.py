@@ -22,7 +22,8 @@ from scipy.stats import norm
 import oracle
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "pages_facts.json")
-FACTS = json.load(open(GOLDEN))
+with open(GOLDEN) as _f:
+    FACTS = json.load(_f)
 
 
 def bits_of(t: torch.Tensor) -> np.ndarray:
