@@ -267,9 +267,11 @@ AQNF4_API int64_t aqnf4_cost_bytes(int64_t n);
    sq_err, sq_w (device double[num_layers], e.g. aqnf4_layer_error's outputs), block_of
    (device int32[num_layers]) and cost_bytes (device int64[num_layers]) are inputs;
    block_rank (device int32[num_blocks]) receives the whole ranking, block_err (optional,
-   device float[num_blocks]) the scores and k_out (device int32[1]) the number of blocks kept,
-   or -1 when a block_of entry lies outside [0, num_blocks) (the other outputs are then
-   meaningless).  1 <= num_blocks <= 2048.  One thread block.
+   device float[num_blocks]) the scores and k_out (device int32[1]) the number of blocks kept.
+   A block_of entry outside [0, num_blocks) is a data error: the kernel stores
+   AQNF4_ERR_INVALID_ARG in *dev_flag (optional device int32, zeroed by the caller) and -1 in
+   *k_out, and the other outputs are then meaningless.  1 <= num_blocks <= 2048.  One thread
+   block.
    Errors: INVALID_ARG (NULL pointer, a size out of range, budget_bytes < 0, unknown order),
    ALIGNMENT, CUDA. */
 enum { AQNF4_BLOCKS_BY_DEPTH = 0, AQNF4_BLOCKS_BY_ERROR = 1 };
@@ -278,7 +280,8 @@ AQNF4_API aqnf4_status aqnf4_select_blocks(const double* sq_err, const double* s
                                            int32_t num_layers, int32_t num_blocks,
                                            int64_t budget_bytes, int32_t order,
                                            int32_t* block_rank, float* block_err,
-                                           int32_t* k_out, cudaStream_t stream);
+                                           int32_t* k_out, int32_t* dev_flag,
+                                           cudaStream_t stream);
 
 /* The fused pass's code lookup, for inspection (host only; no counterpart on the pages,
    which define the code as the nearest level, i.e. the number of midpoints below v).

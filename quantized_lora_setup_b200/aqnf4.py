@@ -101,7 +101,7 @@ def library() -> ctypes.CDLL:
     lib.aqnf4_nf4_linear.restype = st
     lib.aqnf4_nf4_linear_workspace_size.argtypes = [i64, i64, i64]
     lib.aqnf4_nf4_linear_workspace_size.restype = ctypes.c_size_t
-    lib.aqnf4_select_blocks.argtypes = [P, P, P, P, i32, i32, i64, i32, P, P, P, P]
+    lib.aqnf4_select_blocks.argtypes = [P, P, P, P, i32, i32, i64, i32, P, P, P, P, P]
     lib.aqnf4_select_blocks.restype = st
     lib.aqnf4_slot_tables.argtypes = [P, P, P]
     lib.aqnf4_slot_tables.restype = st
@@ -339,7 +339,8 @@ def aqnf4_nf4_linear_workspace_size(M: int, N: int, K: int) -> int:
 def aqnf4_select_blocks(sq_err: torch.Tensor, sq_w: torch.Tensor, block_of: torch.Tensor,
                         cost_bytes: torch.Tensor, num_blocks: int, budget_bytes: int, order: int,
                         block_rank: torch.Tensor, block_err: Optional[torch.Tensor],
-                        k_out: torch.Tensor, stream=None) -> None:
+                        k_out: torch.Tensor, stream=None,
+                        dev_flag: Optional[torch.Tensor] = None) -> None:
     L = sq_err.numel()
     _req(sq_err, "sq_err", (torch.float64,))
     _req(sq_w, "sq_w", (torch.float64,), L)
@@ -348,10 +349,12 @@ def aqnf4_select_blocks(sq_err: torch.Tensor, sq_w: torch.Tensor, block_of: torc
     _req(block_rank, "block_rank", (torch.int32,), num_blocks)
     _req(block_err, "block_err", (torch.float32,), num_blocks, optional=True)
     _req(k_out, "k_out", (torch.int32,), 1)
+    _req(dev_flag, "dev_flag", (torch.int32,), 1, optional=True)
     _check(library().aqnf4_select_blocks(_ptr(sq_err), _ptr(sq_w), _ptr(block_of),
                                          _ptr(cost_bytes), sq_err.numel(), num_blocks,
                                          budget_bytes, order, _ptr(block_rank), _ptr(block_err),
-                                         _ptr(k_out), _stream(stream)), "aqnf4_select_blocks")
+                                         _ptr(k_out), _ptr(dev_flag), _stream(stream)),
+           "aqnf4_select_blocks")
 
 
 def aqnf4_slot_tables():

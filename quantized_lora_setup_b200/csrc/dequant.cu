@@ -11,15 +11,21 @@
 // consecutive chunks, so loads and stores are fully coalesced; a warp-iteration covers
 // 8 x 32 chunks for memory-level parallelism.  The level lookup is a warp shuffle whose
 // source lane is the nibble itself (lanes 16..31 mirror 0..15, so the shifted word needs
-// no mask).  fl(c / 255) for the 256 possible bytes is tabulated in shared memory with a
-// correctly rounded divide.  Stores are streaming (evict-first), which the write-heavy
+// no mask).  fl(c / 255) for the 256 possible bytes is tabulated in shared memory (the
+// short exact quotient of device.cuh).  Stores are streaming (evict-first), which the write-heavy
 // traffic favours.
 #include "device.cuh"
 
 namespace aqnf4 {
 namespace {
 
-constexpr int kChunksPerLane = 8;  // 16 costs occupancy (108 registers), 4 too few loads in flight
+#ifndef AQNF4_DQ_CHUNKS
+#define AQNF4_DQ_CHUNKS 8
+#endif
+#ifndef AQNF4_DQ_OCC_GRID
+#define AQNF4_DQ_OCC_GRID 0
+#endif
+constexpr int kChunksPerLane = AQNF4_DQ_CHUNKS;  // 16 costs occupancy (108 registers)
 
 struct DqParams {
   float level[16];
@@ -35,7 +41,8 @@ __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ pac
   using F = Fmt<DT>;
   __shared__ float frac[256];
   const int t = threadIdx.x, lane = t & 31;
-  frac[t] = __fdiv_rn(static_cast<float>(t), 255.0f);
+  // t and 255 are 16-bit values with t <= 255, where the short quotient is exactly fl(t / 255)
+  frac[t] = quot16_rn(static_cast<float>(t), 255.0f, rcp16_rn(255.0f));
   __syncthreads();
   const float tab_level = p.level[lane & 15];
 
@@ -113,6 +120,12 @@ extern "C" aqnf4_status aqnf4_dequantize(const uint8_t* packed, const uint8_t* c
   const int64_t groups = (nchunk + 32 * kChunksPerLane - 1) / (32 * kChunksPerLane);
   const int sms = current_sm_count();
   int64_t grid = static_cast<int64_t>(sms > 0 ? sms : 1) * 8;  // 8 warps per CTA
+  if (AQNF4_DQ_OCC_GRID) {
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_dequant<AQNF4_BF16>, 256, 0) ==
+            cudaSuccess && occ > 0)
+      grid = static_cast<int64_t>(sms > 0 ? sms : 1) * occ;
+  }
   const int64_t need = (groups + 7) / 8;
   if (grid > need) grid = need;
   uint16_t* o = static_cast<uint16_t*>(out);

@@ -92,7 +92,8 @@ constexpr int kMaxBlocks = 2048;
 __global__ void __launch_bounds__(kSelThreads) k_select_blocks(
     const double* __restrict__ sq_err, const double* __restrict__ sq_w,
     const int32_t* __restrict__ block_of, const int64_t* __restrict__ cost, int L, int B,
-    int64_t budget, int order, int32_t* block_rank, float* block_err, int32_t* k_out) {
+    int64_t budget, int order, int32_t* block_rank, float* block_err, int32_t* k_out,
+    int32_t* flag) {
   __shared__ float s_err[kMaxBlocks];
   __shared__ int64_t s_cost[kMaxBlocks];
   __shared__ int bad;
@@ -132,6 +133,7 @@ __global__ void __launch_bounds__(kSelThreads) k_select_blocks(
     while (k < B && used + s_cost[__ldcg(block_rank + k)] <= budget)
       used += s_cost[__ldcg(block_rank + k++)];
     *k_out = bad ? -1 : k;
+    if (bad && flag) *flag = AQNF4_ERR_INVALID_ARG;
   }
 }
 
@@ -159,18 +161,19 @@ extern "C" aqnf4_status aqnf4_select_blocks(const double* sq_err, const double* 
                                             int32_t num_layers, int32_t num_blocks,
                                             int64_t budget_bytes, int32_t order,
                                             int32_t* block_rank, float* block_err,
-                                            int32_t* k_out, cudaStream_t stream) {
+                                            int32_t* k_out, int32_t* dev_flag,
+                                            cudaStream_t stream) {
   if (!sq_err || !sq_w || !block_of || !cost_bytes || !block_rank || !k_out ||
       num_layers < 1 || num_blocks < 1 || num_blocks > kMaxBlocks || budget_bytes < 0 ||
       (order != AQNF4_BLOCKS_BY_DEPTH && order != AQNF4_BLOCKS_BY_ERROR))
     return AQNF4_ERR_INVALID_ARG;
   if (!is_aligned(sq_err, 8) || !is_aligned(sq_w, 8) || !is_aligned(block_of, 4) ||
       !is_aligned(cost_bytes, 8) || !is_aligned(block_rank, 4) || !is_aligned(block_err, 4) ||
-      !is_aligned(k_out, 4))
+      !is_aligned(k_out, 4) || !is_aligned(dev_flag, 4))
     return AQNF4_ERR_ALIGNMENT;
   k_select_blocks<<<1, kSelThreads, 0, stream>>>(sq_err, sq_w, block_of, cost_bytes, num_layers,
                                                  num_blocks, budget_bytes, order, block_rank,
-                                                 block_err, k_out);
+                                                 block_err, k_out, dev_flag);
   count_launches(1);
   return cudaGetLastError() == cudaSuccess ? AQNF4_OK : AQNF4_ERR_CUDA;
 }

@@ -71,26 +71,41 @@ class SplitModel:
         aqnf4.aqnf4_dequantize(st.packed, st.codes8, st.scales, None, L.numel, out, stream)
         return out
 
+    def linear_path(self, i: int, x_dtype: torch.dtype) -> str:
+        """Which path linear(i, x) takes for an x of the given dtype:
+        "cublas-16bit" (a kept layer), "fused-nf4" (the fused NF4-dequant tensor-core GEMM), or
+        "dequantize+cublas" (an NF4 layer whose K is not a multiple of 64, or an x whose 16-bit
+        format differs from the layer's: the layer is dequantized, x converted to the layer's
+        format, and cuBLAS multiplies)."""
+        L = self.layers[i]
+        if L.kind == "fp16":
+            return "cublas-16bit"
+        if len(L.shape) != 2 or L.shape[1] % 64 != 0 or x_dtype != L.dtype:
+            return "dequantize+cublas"
+        return "fused-nf4"
+
     def linear(self, i: int, x: torch.Tensor, out_dtype: Optional[torch.dtype] = None,
                stream=None) -> torch.Tensor:
-        """The forward product of layer i, y = x w^T, for x (M x K) in the layer's 16-bit
-        format: cuBLAS on the kept 16-bit weights, or the fused NF4-dequant tensor-core GEMM
-        (aqnf4_nf4_linear) on the NF4 + DQ storage.  A layer whose K is not a multiple of 64
-        (rows would not be whole NF4 blocks) is dequantized first and multiplied by cuBLAS."""
+        """The forward product of layer i, y = x w^T, for x (M x K): cuBLAS on the kept 16-bit
+        weights, or the fused NF4-dequant tensor-core GEMM (aqnf4_nf4_linear) on the NF4 + DQ
+        storage.  A layer whose K is not a multiple of 64 (rows would not be whole NF4 blocks),
+        or an x in the other 16-bit format, is dequantized first and multiplied by cuBLAS with
+        x converted to the layer's format; linear_path(i, x.dtype) names the path taken."""
         L = self.layers[i]
         if len(L.shape) != 2:
             raise ValueError("linear: the layer is not a matrix")
         N, K = L.shape
         out_dtype = out_dtype or x.dtype
+        path = self.linear_path(i, x.dtype)
 
         def dense(w16):  # cuBLAS; a float32 result is summed in binary32 without 16-bit rounding
             if out_dtype == torch.float32:
                 return torch.matmul(x.to(L.dtype).float(), w16.float().t())
             return torch.matmul(x.to(L.dtype), w16.t()).to(out_dtype)
 
-        if L.kind == "fp16":
+        if path == "cublas-16bit":
             return dense(L.weight)
-        if K % 64 != 0 or x.dtype != L.dtype:
+        if path == "dequantize+cublas":
             return dense(self.weight(i, stream=stream))
         M = x.shape[0]
         y = torch.empty((M, N), dtype=out_dtype if out_dtype == torch.float32 else x.dtype,

@@ -136,13 +136,16 @@ def test_argument_checks_return_before_any_launch(lib):
     assert lib.aqnf4_select_topk(V(0x100), V(0x204), 5, 10, -1, V(0x300), V(0x400), None) == aqnf4.AQNF4_ERR_ALIGNMENT
     # block selection
     args = [V(0x100), V(0x200), V(0x300), V(0x400), 5, 3, 10, aqnf4.AQNF4_BLOCKS_BY_DEPTH,
-            V(0x500), None, V(0x600), None]
+            V(0x500), None, V(0x600), None, None]
     for i, bad_value in ((0, None), (4, 0), (5, 0), (5, 2049), (6, -1), (7, 2), (10, None)):
         a = list(args)
         a[i] = bad_value
         assert lib.aqnf4_select_blocks(*a) == aqnf4.AQNF4_ERR_INVALID_ARG, (i, bad_value)
     a = list(args)
     a[0] = V(0x104)
+    assert lib.aqnf4_select_blocks(*a) == aqnf4.AQNF4_ERR_ALIGNMENT
+    a = list(args)
+    a[11] = V(0x702)  # dev_flag not 4-byte aligned
     assert lib.aqnf4_select_blocks(*a) == aqnf4.AQNF4_ERR_ALIGNMENT
     # bounded-wait diagnostic
     assert lib.aqnf4_selftest_wait_timeout(0, V(0x100), None, None) == aqnf4.AQNF4_ERR_INVALID_ARG

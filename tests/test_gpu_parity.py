@@ -489,6 +489,14 @@ def test_select_blocks_reports_a_bad_block_index(cuda):
     cost = torch.ones(4, dtype=torch.int64, device=cuda)
     rank = torch.empty(2, dtype=torch.int32, device=cuda)
     k = torch.empty(1, dtype=torch.int32, device=cuda)
+    flag = torch.zeros(1, dtype=torch.int32, device=cuda)
     aqnf4.aqnf4_select_blocks(se, se, block_of, cost, 2, 10, aqnf4.AQNF4_BLOCKS_BY_DEPTH, rank,
-                              None, k)
+                              None, k, dev_flag=flag)
     assert k.item() == -1
+    assert flag.item() == aqnf4.AQNF4_ERR_INVALID_ARG
+    # a valid call leaves the flag word alone
+    flag.zero_()
+    block_of = torch.tensor([0, 1, 1, 1], dtype=torch.int32, device=cuda)
+    aqnf4.aqnf4_select_blocks(se, se, block_of, cost, 2, 10, aqnf4.AQNF4_BLOCKS_BY_DEPTH, rank,
+                              None, k, dev_flag=flag)
+    assert k.item() == 2 and flag.item() == 0

@@ -126,3 +126,33 @@ def test_split_model_linear_matches_oracle(cuda):
         ref = x64 @ w64.T
         bound = K * 2.0 ** -23 * (np.abs(x64) @ np.abs(w64).T) + 1e-30
         assert np.all(np.abs(y - ref) <= bound), i
+
+
+@pytest.mark.gpu
+def test_split_model_linear_dequantize_path_matches_oracle(cuda):
+    """The branch that multiplies dequantized weights: an NF4 layer whose K (100, 72) is not a
+    multiple of 64, so NF4 blocks cross rows, and an x in the other 16-bit format on a layer
+    the fused GEMM could take.  Each result is within the binary32 accumulation bound of the
+    oracle's binary64 product of x (in the layer's format) with the oracle's w_hat."""
+    rng = np.random.default_rng(43)
+    shapes = [(160, 100), (96, 72), (128, 128)]
+    weights = [torch.from_numpy((rng.standard_normal(sh) * 0.02).astype(np.float32))
+               .to(torch.bfloat16).to(cuda) for sh in shapes]
+    model = split_model.materialize(weights, budget_bytes=0)  # every layer stays NF4
+    assert all(L.kind == "nf4" for L in model.layers)
+    M = 40
+    cases = [(0, torch.bfloat16), (1, torch.bfloat16), (2, torch.float16), (2, torch.bfloat16)]
+    for i, x_dtype in cases:
+        N, K = shapes[i]
+        want = "fused-nf4" if (K % 64 == 0 and x_dtype == torch.bfloat16) else \
+            "dequantize+cublas"
+        assert model.linear_path(i, x_dtype) == want, (i, x_dtype)
+        x = torch.from_numpy(rng.standard_normal((M, K)).astype(np.float32)).to(x_dtype)
+        y = model.linear(i, x.to(cuda), out_dtype=torch.float32).double().cpu().numpy()
+        xl = x.to(torch.bfloat16)  # x as the product sees it: in the layer's format
+        packed, absmax, _ = oracle.quantize(synth.bits_u16(weights[i].cpu()), oracle.BF16)
+        codes8, scales, _ = oracle.double_quant(absmax)
+        ref, rabs = oracle.nf4_linear(synth.bits_u16(xl).reshape(M, K), oracle.BF16, packed,
+                                      codes8, scales, N, oracle.BF16)
+        bound = K * 2.0 ** -23 * rabs + 1e-30
+        assert np.all(np.abs(y - ref) <= bound), (i, x_dtype)
