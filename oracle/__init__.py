@@ -47,6 +47,12 @@ def load():
     lib.oracle_double_quant.restype = None
     lib.oracle_dequantize.argtypes = [P, P, P, P, i64, ctypes.c_int, P, P]
     lib.oracle_dequantize.restype = None
+    lib.oracle_double_quant_centered.argtypes = [P, i64, P, P, P, P]
+    lib.oracle_double_quant_centered.restype = None
+    lib.oracle_dequantize_centered.argtypes = [P, P, P, P, i64, ctypes.c_int, P, P]
+    lib.oracle_dequantize_centered.restype = None
+    lib.oracle_layer_error_dqc.argtypes = [P, ctypes.c_int, i64, P, P, P, P, P]
+    lib.oracle_layer_error_dqc.restype = ctypes.c_int
     lib.oracle_cost_bytes.argtypes = [i64]
     lib.oracle_cost_bytes.restype = i64
     lib.oracle_select_topk.argtypes = [P, P, ctypes.c_int, i64, ctypes.c_int, P, P]
@@ -222,3 +228,43 @@ __all__ = ["F16", "BF16", "load", "default_pmax", "codebook", "quantize", "layer
            "double_quant", "dequantize", "cost_bytes", "select_topk", "f32_to_dtype_bits",
            "dtype_bits_to_f32"]
 
+
+
+def double_quant_centered(absmax):
+    """(codes8 uint8[nb], scales float32[nd], means float32[nd], nonfinite) of the mean-centred
+    8-bit double quantization of the binary32 block constants."""
+    a = np.ascontiguousarray(absmax, np.float32)
+    nb = a.size
+    nd = (nb + 255) // 256
+    codes8 = np.zeros(nb, np.uint8)
+    scales = np.zeros(nd, np.float32)
+    means = np.zeros(nd, np.float32)
+    bad = ctypes.c_int(0)
+    load().oracle_double_quant_centered(_ptr(a), nb, _ptr(codes8), _ptr(scales), _ptr(means),
+                                        ctypes.byref(bad))
+    return codes8, scales, means, bool(bad.value)
+
+
+def dequantize_centered(packed, n: int, out_dtype, codes8, scales, means, book=None):
+    """uint16[n] 16-bit bit patterns of the NF4 tensor rebuilt from mean-centred DQ storage."""
+    levels, _ = book if book is not None else codebook()
+    out = np.zeros(n, np.uint16)
+    load().oracle_dequantize_centered(_ptr(np.ascontiguousarray(packed, np.uint8)),
+                                      _ptr(np.ascontiguousarray(codes8, np.uint8)),
+                                      _ptr(np.ascontiguousarray(scales, np.float32)),
+                                      _ptr(np.ascontiguousarray(means, np.float32)), n,
+                                      out_dtype, _ptr(levels), _ptr(out))
+    return out
+
+
+def layer_error_dqc(w, dtype, book=None):
+    """(sq_err, sq_w, rel_err) of one layer stored in NF4 with mean-centred DQ."""
+    w = _as_bits(w).reshape(-1)
+    levels, mids = book if book is not None else codebook()
+    se = np.zeros(1, np.float64)
+    sw = np.zeros(1, np.float64)
+    rel = np.zeros(1, np.float32)
+    if load().oracle_layer_error_dqc(_ptr(w), dtype, w.size, _ptr(levels), _ptr(mids), _ptr(se),
+                                     _ptr(sw), _ptr(rel)) != 0:
+        raise MemoryError("oracle_layer_error_dqc")
+    return float(se[0]), float(sw[0]), float(rel[0])

@@ -49,6 +49,9 @@
  *     double-quantized constant a' = fl(fl(code8/255) * s) -- what a stored NF4 + DQ model
  *     dequantizes to -- while the codes still come from the binary32 absmax.
  *   - linear layer on NF4 weights: y = x w_hat^T in binary64, w_hat rebuilt as dequantize does.
+ *   - mean-centred DQ (an option, from outside the pages): per 256 constants the binary64
+ *     tree-sum mean mu, h = max |a - mu|, q = rint_even(fl(fl((a - mu)/h) * 127)) stored as
+ *     q + 128, rebuilt as fl(fl(fl(q/127) * h) + mu).
  *   - selection: sort by (score desc, index asc, NaN last); keep the longest prefix with
  *     at most k_cap layers and total incremental cost <= budget.
  */
@@ -326,6 +329,133 @@ void oracle_double_quant(const float* absmax, int64_t nb, uint8_t* codes8, float
       codes8[start + i] = (uint8_t)c;
     }
   }
+}
+
+/* ------------------------------------------------ mean-centred double quantization */
+
+/* A second, optional DQ format ([QLoRA/HIW] gives only the 0.37-bit saving; centring the
+   constants on their mean before a symmetric 8-bit code is a reading from outside the
+   pages).  Per block of 256 constants (the last block may hold only len of them):
+   (1) S = their sum in binary64 over a balanced binary tree of the 256 slots in index
+       order (slot i + 1 pairs with slot i first, then pairs of pairs ...; the missing
+       slots of a short block hold +0);
+   (2) mean mu = fl32(fl64(S / len));
+   (3) c_i = fl(a_i - mu); h = max |c_i|;
+   (4) q_i = rint_even(fl(fl(c_i / h) * 127)) in [-127, 127], stored code8 = q_i + 128
+       (h = 0: every code 128);
+   (5) the constant a dequantization rebuilds: a'_i = fl(fl(fl(q_i / 127) * h) + mu).
+   Storage per block: 256 codes, h and mu: 8/64 + 64/(64*256) = 0.12890625 bits per weight,
+   0.37109375 less than binary32 constants.  A NaN or infinite constant makes the block's
+   mu or h non-finite: its codes are 0, h and mu are stored as computed, *nonfinite set. */
+static double or_tree_sum(const double* v, int n) { /* n a power of two */
+  if (n == 1) return v[0];
+  return or_tree_sum(v, n / 2) + or_tree_sum(v + n / 2, n / 2);
+}
+
+void oracle_double_quant_centered(const float* absmax, int64_t nb, uint8_t* codes8,
+                                  float* scales, float* means, int* nonfinite) {
+  int64_t nd = (nb + OR_DQ_BLOCK - 1) / OR_DQ_BLOCK;
+  double slot[OR_DQ_BLOCK];
+  for (int64_t d = 0; d < nd; ++d) {
+    int64_t start = d * OR_DQ_BLOCK;
+    int64_t len = nb - start < OR_DQ_BLOCK ? nb - start : OR_DQ_BLOCK;
+    for (int64_t i = 0; i < OR_DQ_BLOCK; ++i) slot[i] = i < len ? (double)absmax[start + i] : 0.0;
+    double S = or_tree_sum(slot, OR_DQ_BLOCK);
+    float mu = (float)(S / (double)len);
+    float h = 0.0f;
+    for (int64_t i = 0; i < len; ++i) {
+      float c = fabsf(absmax[start + i] - mu);
+      if (isnan(c) || c > h) h = c;
+    }
+    scales[d] = h;
+    means[d] = mu;
+    if (!isfinite(mu) || !isfinite(h)) {
+      if (nonfinite) *nonfinite = 1;
+      for (int64_t i = 0; i < len; ++i) codes8[start + i] = 0;
+      continue;
+    }
+    for (int64_t i = 0; i < len; ++i) {
+      if (h == 0.0f) {
+        codes8[start + i] = 128;
+        continue;
+      }
+      float c = absmax[start + i] - mu;
+      float t = c / h; /* correctly rounded divide */
+      float q = nearbyintf(t * 127.0f);
+      codes8[start + i] = (uint8_t)(int)(q + 128.0f);
+    }
+  }
+}
+
+/* The constant block b rebuilds from mean-centred DQ storage (step 5 above). */
+static float or_centered_constant(const uint8_t* codes8, const float* scales,
+                                  const float* means, int64_t b) {
+  float t = (float)((int)codes8[b] - 128) / 127.0f;
+  float u = t * scales[b / OR_DQ_BLOCK];
+  return u + means[b / OR_DQ_BLOCK];
+}
+
+/* NF4 -> 16-bit from mean-centred DQ storage: as oracle_dequantize with the constant of
+   or_centered_constant. */
+void oracle_dequantize_centered(const uint8_t* packed, const uint8_t* codes8,
+                                const float* scales, const float* means, int64_t n,
+                                int out_dtype, const float levels[16], uint16_t* out) {
+  for (int64_t e = 0; e < n; ++e) {
+    float a = or_centered_constant(codes8, scales, means, e / OR_BLOCK);
+    uint8_t byte = packed[e >> 1];
+    int code = (e & 1) == 0 ? (byte >> 4) : (byte & 15);
+    out[e] = or_round_to_dtype(levels[code] * a, out_dtype);
+  }
+}
+
+/* The layer error of a model stored in NF4 with mean-centred DQ: as oracle_layer_error_dq
+   with the constant of or_centered_constant.  Returns 0, or -1 if memory runs out. */
+int oracle_layer_error_dqc(const uint16_t* w, int dtype, int64_t n, const float levels[16],
+                           const float mids[15], double* sq_err, double* sq_w, float* rel) {
+  int64_t nb = (n + OR_BLOCK - 1) / OR_BLOCK;
+  int64_t nd = (nb + OR_DQ_BLOCK - 1) / OR_DQ_BLOCK;
+  float* absmax = (float*)calloc((size_t)nb, sizeof(float));
+  uint8_t* codes8 = (uint8_t*)calloc((size_t)nb, 1);
+  float* scales = (float*)calloc((size_t)nd, sizeof(float));
+  float* means = (float*)calloc((size_t)nd, sizeof(float));
+  if (!absmax || !codes8 || !scales || !means) {
+    free(absmax);
+    free(codes8);
+    free(scales);
+    free(means);
+    return -1;
+  }
+  for (int64_t b = 0; b < nb; ++b) {
+    int64_t start = b * OR_BLOCK;
+    int len = (int)(n - start < OR_BLOCK ? n - start : OR_BLOCK);
+    absmax[b] = or_block_absmax(w, dtype, start, len);
+  }
+  oracle_double_quant_centered(absmax, nb, codes8, scales, means, NULL);
+  int codes[OR_BLOCK];
+  double se = 0.0, sw = 0.0;
+  for (int64_t b = 0; b < nb; ++b) {
+    int64_t start = b * OR_BLOCK;
+    int len = (int)(n - start < OR_BLOCK ? n - start : OR_BLOCK);
+    float a_dq = or_centered_constant(codes8, scales, means, b);
+    or_block_codes(w, dtype, start, len, absmax[b], mids, codes);
+    for (int i = 0; i < len; ++i) {
+      float x = or_load(w[start + i], dtype);
+      float what = or_load(or_round_to_dtype(levels[codes[i]] * a_dq, dtype), dtype);
+      double d = (double)x - (double)what;
+      se += d * d;
+      sw += (double)x * (double)x;
+    }
+  }
+  free(absmax);
+  free(codes8);
+  free(scales);
+  free(means);
+  *sq_err = se;
+  *sq_w = sw;
+  double e = sw == 0.0 ? 0.0 : sqrt(se / sw);
+  if (isnan(se) || isnan(sw)) e = NAN;
+  *rel = (float)e;
+  return 0;
 }
 
 /* ------------------------------------------------ DQ-absmax layer error */

@@ -393,6 +393,119 @@ def test_dq_codes_equal_bruteforce_nearest():
             assert np.all(np.abs(frac - np.floor(frac) - 0.5) < 1e-5)
 
 
+def test_dqc_saving_matches_page_figure():
+    """Mean-centred DQ stores 8-bit codes plus two binary32 numbers per 256 constants:
+    8/64 + 64/(64*256) bits per weight, 0.37109375 less than binary32 constants -- the pages'
+    0.37 bits as well ("QLoRA", How It Works)."""
+    n = 64 * 256 * 10
+    absmax = np.random.default_rng(0).uniform(0, 1, n // 64).astype(np.float32)
+    codes8, scales, means, _ = oracle.double_quant_centered(absmax)
+    bits = (codes8.nbytes + scales.nbytes + means.nbytes) * 8 / n
+    saving = absmax.nbytes * 8 / n - bits
+    assert saving == 0.5 - (8 / 64 + 64 / (64 * 256)) == 0.37109375
+    fact = FACTS["dq_saving_bits_per_param"]
+    assert round(saving, fact["decimals"]) == fact["value"]
+
+
+def test_dqc_mean_is_the_exact_mean():
+    """For 16-bit constants a few binades apart the binary64 tree sum is exact, so the mean
+    is the exact rational mean rounded to binary64, then to binary32 (also for a short
+    last block)."""
+    from fractions import Fraction
+    rng = np.random.default_rng(5)
+    for nb in (256 * 3, 256 * 2 + 37):
+        a = torch.from_numpy(np.abs(rng.standard_normal(nb) * 0.03).astype(np.float32)) \
+            .to(torch.bfloat16).float().numpy()
+        _, _, means, _ = oracle.double_quant_centered(a)
+        for d in range(means.size):
+            blk = a[256 * d: 256 * d + 256]
+            exact = sum(Fraction(float(v)) for v in blk) / blk.size
+            assert means[d] == np.float32(float(exact)), d
+
+
+def test_dqc_codes_equal_bruteforce_nearest():
+    """Each code is the nearest of the 255 rebuildable offsets fl(fl(q/127) h), q in
+    [-127, 127], to a - mu, except within one rounding of a half-way point."""
+    rng = np.random.default_rng(6)
+    a = np.abs(rng.standard_normal(256 * 29 + 11)).astype(np.float32) * 0.05
+    codes8, scales, means, _ = oracle.double_quant_centered(a)
+    q = np.arange(-127, 128)
+    for d in range(scales.size):
+        blk = a[256 * d: 256 * d + 256]
+        h, mu = scales[d], means[d]
+        c = (blk - mu).astype(np.float32).astype(np.float64)
+        assert h == np.abs(c).max()
+        grid = ((q.astype(np.float32) / np.float32(127)) * h).astype(np.float64)
+        brute = q[np.argmin(np.abs(c[:, None] - grid[None, :]), axis=1)]
+        got = codes8[256 * d: 256 * d + blk.size].astype(np.int64) - 128
+        diff = got != brute
+        assert diff.sum() <= 2
+        if diff.any():
+            t = c[diff] / h * 127
+            assert np.all(np.abs(t - np.floor(t) - 0.5) < 1e-4)
+
+
+def test_dqc_special_blocks():
+    """A block of one repeated value rebuilds it exactly (h = 0, codes 128); a block of two
+    values symmetric about their mean codes to the ends 1 and 255 and rebuilds both
+    exactly; a non-finite constant is flagged."""
+    v = np.float32(0.0375)
+    codes8, scales, means, nf = oracle.double_quant_centered(np.full(256, v, np.float32))
+    assert not nf and scales[0] == 0 and means[0] == v and np.all(codes8 == 128)
+    lo, hi = np.float32(0.25), np.float32(0.75)
+    a = np.array([lo, hi] * 128, np.float32)
+    codes8, scales, means, _ = oracle.double_quant_centered(a)
+    assert means[0] == 0.5 and scales[0] == 0.25
+    assert list(codes8[:2]) == [1, 255]
+    rebuilt = (((codes8.astype(np.int32) - 128).astype(np.float32) / np.float32(127))
+               * scales[0] + means[0]).astype(np.float32)
+    assert np.array_equal(rebuilt, a)
+    _, _, _, nf = oracle.double_quant_centered(np.array([1.0, np.inf], np.float32))
+    assert nf
+
+
+def test_dqc_rebuilt_constants_are_closer_for_clustered_constants(book):
+    """Centring on the mean spends the 8-bit code on [mu - h, mu + h] instead of [0, s]: for
+    the absmax values of normal 64-blocks (mean about 2.4 sigma, spread about as wide) the
+    code's step is about 3/4 of the plain code's, so the rebuilt constants land closer on
+    average, each within h/254 plus rounding."""
+    rng = np.random.default_rng(7)
+    w = torch.from_numpy((rng.standard_normal(64 * 256 * 8) * 0.02).astype(np.float32)) \
+        .to(torch.bfloat16)
+    _, absmax, _ = oracle.quantize(bits_of(w), oracle.BF16)
+    c8, sc, mu, _ = oracle.double_quant_centered(absmax)
+    rc = (((c8.astype(np.int32) - 128).astype(np.float32) / np.float32(127))
+          * np.repeat(sc, 256) + np.repeat(mu, 256)).astype(np.float32)
+    p8, ps, _ = oracle.double_quant(absmax)
+    rp = ((p8.astype(np.float32) / np.float32(255)) * np.repeat(ps, 256)).astype(np.float32)
+    err_c = np.abs(rc.astype(np.float64) - absmax)
+    err_p = np.abs(rp.astype(np.float64) - absmax)
+    assert err_c.mean() < 0.85 * err_p.mean()
+    assert np.all(err_c <= np.repeat(sc, 256) / 254 * (1 + 1e-5) + 4e-7 * absmax)
+
+
+@pytest.mark.parametrize("dtype", [oracle.F16, oracle.BF16])
+def test_dqc_layer_error_is_the_error_of_the_dequantized_model(book, dtype):
+    """The layer error against mean-centred DQ constants equals the error of what the
+    centred dequantization rebuilds, summed here in numpy (3 DQ blocks, ragged tail)."""
+    rng = np.random.default_rng(23)
+    n = 64 * 700 + 13
+    tdt = torch.float16 if dtype == oracle.F16 else torch.bfloat16
+    z = rng.standard_normal(n) * np.repeat(rng.uniform(0.005, 0.05, n // 64 + 1), 64)[:n]
+    w = torch.from_numpy(z.astype(np.float32)).to(tdt)
+    bits = bits_of(w)
+    packed, absmax, _ = oracle.quantize(bits, dtype)
+    codes8, scales, means, _ = oracle.double_quant_centered(absmax)
+    deq = oracle.dequantize_centered(packed, n, dtype, codes8, scales, means)
+    deq = torch.from_numpy(deq.view(np.int16)).view(tdt).double().numpy()
+    x = w.double().numpy()
+    se, sw, rel = oracle.layer_error_dqc(bits, dtype)
+    assert se == pytest.approx(float(np.sum((x - deq) ** 2)), rel=1e-12)
+    assert sw == oracle.layer_error(bits, dtype)[1]
+    assert rel == pytest.approx(math.sqrt(se / sw), rel=1e-6)
+    assert se != oracle.layer_error_dq(bits, dtype)[0]
+
+
 def test_dequant_with_exact_dq_equals_plain_absmax(book):
     """Constants that double-quantize exactly (code 255) dequantize like the raw absmax."""
     rng = np.random.default_rng(8)
