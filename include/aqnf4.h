@@ -79,7 +79,13 @@ enum {
      a'_b = fl(fl(code8_b / 255) * s) of its block, exactly what aqnf4_dequantize returns
      from packed + codes8 + scales, instead of the binary32 absmax a_b.  The codes, packed
      bytes, absmax, codes8 and scales written are the same either way. */
-  AQNF4_SCORE_DQ_ABSMAX = 1
+  AQNF4_SCORE_DQ_ABSMAX = 1,
+  /* Score the layer as NF4 with mean-centred double quantization would store it
+     (aqnf4_double_quant_centered, a format from outside the pages): w_hat is rebuilt from
+     a'_b = fl(fl(fl((code8_b - 128) / 127) * h) + mu) of its DQ block, exactly what
+     aqnf4_dequantize_centered returns.  The stored outputs are still the plain format's.
+     At most one of the two score flags may be set. */
+  AQNF4_SCORE_DQ_CENTERED = 2
 };
 
 /* One linear layer for aqnf4_layer_error.  All pointers are device pointers.
@@ -148,6 +154,33 @@ AQNF4_API aqnf4_status aqnf4_dequantize(const uint8_t* packed, const uint8_t* co
                               const float* scales, const float* absmax, int64_t n,
                               int32_t out_dtype, void* out, cudaStream_t stream);
 
+/* Mean-centred double quantization, a second storage format for the block constants.  The
+   pages give only the 0.37-bit saving ("QLoRA", "How It Works"); centring the constants on
+   their mean before a symmetric 8-bit code is a reading from outside them, offered as an
+   option beside aqnf4_double_quant.  Per block of 256 constants (the last may be short,
+   len of them): S = their binary64 sum over a balanced binary tree of the 256 slots in index
+   order (missing slots hold +0); mean mu = fl32(fl64(S / len)); h = max |fl(a - mu)|;
+   code8 = rint_even(fl(fl(fl(a - mu) / h) * 127)) + 128 in [1, 255] (h = 0: 128).  The
+   constant rebuilt is a' = fl(fl(fl((code8 - 128) / 127) * h) + mu).  Storage: 8/64 +
+   64/(64*256) bits per weight (0.371 below binary32 constants).
+   absmax (device, 4-byte aligned, nb floats) in; codes8 (device, nb bytes), scales = h and
+   means = mu (device, 4-byte aligned, ceil(nb/256) floats each) out.  A NaN or infinite
+   constant makes its block's mu or h non-finite: the block's codes are 0 and dev_flag
+   (optional) receives AQNF4_ERR_NONFINITE.
+   Errors: INVALID_ARG (NULL pointer, nb < 1), ALIGNMENT, CUDA. */
+AQNF4_API aqnf4_status aqnf4_double_quant_centered(const float* absmax, int64_t nb,
+                                                   uint8_t* codes8, float* scales, float* means,
+                                                   int32_t* dev_flag, cudaStream_t stream);
+
+/* NF4 -> 16-bit dequantization from mean-centred DQ storage (aqnf4_double_quant_centered):
+   as aqnf4_dequantize with the block constant a' = fl(fl(fl((code8 - 128) / 127) *
+   scales[b/256]) + means[b/256]).  All pointers required; packed and out 16-byte aligned,
+   scales and means 4-byte aligned.  Errors: INVALID_ARG, ALIGNMENT, DTYPE, CUDA. */
+AQNF4_API aqnf4_status aqnf4_dequantize_centered(const uint8_t* packed, const uint8_t* codes8,
+                                                 const float* scales, const float* means,
+                                                 int64_t n, int32_t out_dtype, void* out,
+                                                 cudaStream_t stream);
+
 /* Bytes of device workspace aqnf4_layer_error needs for these layers (host only; 0 when
    the arguments are invalid). */
 AQNF4_API size_t aqnf4_workspace_size(const aqnf4_layer* layers, int32_t num_layers);
@@ -157,7 +190,8 @@ AQNF4_API size_t aqnf4_workspace_size(const aqnf4_layer* layers, int32_t num_lay
    layers: HOST array of num_layers descriptors (device pointers inside).  Each layer is
    quantized as in aqnf4_quantize; its optional outputs (packed, absmax, codes8 + scales)
    are written; and, with w_hat = dtype_rn(fl(levels[code] * a_b)) (a_b replaced by the
-   double-quantized a'_b for a layer flagged AQNF4_SCORE_DQ_ABSMAX),
+   double-quantized a'_b for a layer flagged AQNF4_SCORE_DQ_ABSMAX or
+   AQNF4_SCORE_DQ_CENTERED),
      sq_err[l] = sum (x - w_hat)^2,  sq_w[l] = sum x^2,
      rel_err[l] = sqrt(sq_err[l] / sq_w[l])  (0 when sq_w[l] = 0; NaN after a NaN/inf input).
    The sums are taken in a fixed order, so repeated calls give identical bits.

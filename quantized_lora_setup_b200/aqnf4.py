@@ -28,6 +28,7 @@ AQNF4_ERR_WORKSPACE = 7
 AQNF4_F16 = 0
 AQNF4_BF16 = 1
 AQNF4_SCORE_DQ_ABSMAX = 1  # aqnf4_layer.flags
+AQNF4_SCORE_DQ_CENTERED = 2
 AQNF4_BLOCKS_BY_DEPTH = 0  # aqnf4_select_blocks orders
 AQNF4_BLOCKS_BY_ERROR = 1
 
@@ -84,6 +85,10 @@ def library() -> ctypes.CDLL:
     lib.aqnf4_double_quant.restype = st
     lib.aqnf4_dequantize.argtypes = [P, P, P, P, i64, i32, P, P]
     lib.aqnf4_dequantize.restype = st
+    lib.aqnf4_double_quant_centered.argtypes = [P, i64, P, P, P, P, P]
+    lib.aqnf4_double_quant_centered.restype = st
+    lib.aqnf4_dequantize_centered.argtypes = [P, P, P, P, i64, i32, P, P]
+    lib.aqnf4_dequantize_centered.restype = st
     lib.aqnf4_workspace_size.argtypes = [P, i32]
     lib.aqnf4_workspace_size.restype = ctypes.c_size_t
     lib.aqnf4_layer_error.argtypes = [P, i32, P, ctypes.c_size_t, P, P, P, P, P]
@@ -216,6 +221,35 @@ def aqnf4_dequantize(packed: torch.Tensor, codes8: Optional[torch.Tensor],
     _check(library().aqnf4_dequantize(_ptr(packed), _ptr(codes8), _ptr(scales), _ptr(absmax), n,
                                       dtype_code(out.dtype), _ptr(out), _stream(stream)),
            "aqnf4_dequantize")
+
+
+def aqnf4_double_quant_centered(absmax: torch.Tensor, codes8: torch.Tensor,
+                                scales: torch.Tensor, means: torch.Tensor,
+                                dev_flag: Optional[torch.Tensor] = None, stream=None) -> None:
+    nb = absmax.numel()
+    nd = (nb + DQ_BLOCK - 1) // DQ_BLOCK
+    _req(absmax, "absmax", (torch.float32,))
+    _req(codes8, "codes8", (torch.uint8,), nb)
+    _req(scales, "scales", (torch.float32,), nd)
+    _req(means, "means", (torch.float32,), nd)
+    _req(dev_flag, "dev_flag", (torch.int32,), 1, optional=True)
+    _check(library().aqnf4_double_quant_centered(_ptr(absmax), nb, _ptr(codes8), _ptr(scales),
+                                                 _ptr(means), _ptr(dev_flag), _stream(stream)),
+           "aqnf4_double_quant_centered")
+
+
+def aqnf4_dequantize_centered(packed: torch.Tensor, codes8: torch.Tensor, scales: torch.Tensor,
+                              means: torch.Tensor, n: int, out: torch.Tensor,
+                              stream=None) -> None:
+    npk, nb, nsc = _storage_sizes(n)
+    _req(packed, "packed", (torch.uint8,), npk)
+    _req(codes8, "codes8", (torch.uint8,), nb)
+    _req(scales, "scales", (torch.float32,), nsc)
+    _req(means, "means", (torch.float32,), nsc)
+    _req(out, "out", None, n)
+    _check(library().aqnf4_dequantize_centered(_ptr(packed), _ptr(codes8), _ptr(scales),
+                                               _ptr(means), n, dtype_code(out.dtype), _ptr(out),
+                                               _stream(stream)), "aqnf4_dequantize_centered")
 
 
 def make_layers(layers: Sequence[dict]):
@@ -406,6 +440,17 @@ def double_quant(absmax: torch.Tensor, stream=None):
     return codes8, scales
 
 
+def double_quant_centered(absmax: torch.Tensor, stream=None):
+    """(codes8, scales, means) of the mean-centred double quantization."""
+    nb = absmax.numel()
+    nd = (nb + DQ_BLOCK - 1) // DQ_BLOCK
+    codes8 = torch.empty(nb, dtype=torch.uint8, device=absmax.device)
+    scales = torch.empty(nd, dtype=torch.float32, device=absmax.device)
+    means = torch.empty(nd, dtype=torch.float32, device=absmax.device)
+    aqnf4_double_quant_centered(absmax, codes8, scales, means, None, stream)
+    return codes8, scales, means
+
+
 def dequantize(packed: torch.Tensor, n: int, dtype: torch.dtype = torch.bfloat16,
                codes8=None, scales=None, absmax=None, stream=None) -> torch.Tensor:
     out = torch.empty(n, dtype=dtype, device=packed.device)
@@ -426,14 +471,18 @@ class NF4Storage:
 
 
 def score_layers(weights: List[torch.Tensor], storages: Optional[List[NF4Storage]] = None,
-                 stream=None, dq_score: bool = False):
+                 stream=None, dq_score=False):
     """Run the fused quantize+score pass: returns (sq_err f64[L], sq_w f64[L], rel_err f32[L]).
-    dq_score: score against the double-quantized constants (AQNF4_SCORE_DQ_ABSMAX)."""
+    dq_score: score against the double-quantized constants -- True or "absmax" for the
+    plain 8-bit DQ (AQNF4_SCORE_DQ_ABSMAX), "centered" for mean-centred DQ
+    (AQNF4_SCORE_DQ_CENTERED)."""
     dev = weights[0].device
     L = len(weights)
+    flags = {False: 0, None: 0, True: AQNF4_SCORE_DQ_ABSMAX, "absmax": AQNF4_SCORE_DQ_ABSMAX,
+             "centered": AQNF4_SCORE_DQ_CENTERED}[dq_score]
     descs = []
     for i, w in enumerate(weights):
-        d = {"w": w, "flags": AQNF4_SCORE_DQ_ABSMAX if dq_score else 0}
+        d = {"w": w, "flags": flags}
         if storages is not None:
             s = storages[i]
             d.update(packed=s.packed, codes8=s.codes8, scales=s.scales, absmax=s.absmax)

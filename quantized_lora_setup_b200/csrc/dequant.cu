@@ -19,19 +19,17 @@
 namespace aqnf4 {
 namespace {
 
-#ifndef AQNF4_DQ_CHUNKS
-#define AQNF4_DQ_CHUNKS 8
-#endif
-#ifndef AQNF4_DQ_OCC_GRID
-#define AQNF4_DQ_OCC_GRID 0
-#endif
-constexpr int kChunksPerLane = AQNF4_DQ_CHUNKS;  // 16 costs occupancy (108 registers)
+// 16 chunks per lane cost occupancy (108 registers); 2 or 4 measured slower from 16 MB up
+constexpr int kChunksPerLane = 8;
 
 struct DqParams {
   float level[16];
 };
 
-template <int DT>
+// CENTERED: the constants come from mean-centred DQ storage, a' = fl(fl(fl(q/127) * h) + mu)
+// with q = code8 - 128, h = scales[b / 256] and mu = means[b / 256] (`absmax` carries the
+// means); otherwise a' = fl(fl(code8/255) * s), or the plain absmax when codes8 is NULL.
+template <int DT, bool CENTERED>
 __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ packed,
                                                  const uint8_t* __restrict__ codes8,
                                                  const float* __restrict__ scales,
@@ -41,8 +39,10 @@ __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ pac
   using F = Fmt<DT>;
   __shared__ float frac[256];
   const int t = threadIdx.x, lane = t & 31;
-  // t and 255 are 16-bit values with t <= 255, where the short quotient is exactly fl(t / 255)
-  frac[t] = quot16_rn(static_cast<float>(t), 255.0f, rcp16_rn(255.0f));
+  if (CENTERED)
+    frac[t] = __fdiv_rn(static_cast<float>(t - 128), 127.0f);
+  else  // t and 255 are 16-bit values, t <= 255: the short quotient is exactly fl(t / 255)
+    frac[t] = quot16_rn(static_cast<float>(t), 255.0f, rcp16_rn(255.0f));
   __syncthreads();
   const float tab_level = p.level[lane & 15];
 
@@ -69,8 +69,12 @@ __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ pac
       }
       if (c < nchunk) {
         const int64_t b = c >> 3;  // 8 chunks per 64-element block
-        ap[j] = codes8 ? __fmul_rn(frac[__ldg(codes8 + b)], __ldg(scales + (b >> 8)))
-                       : __ldg(absmax + b);
+        if (CENTERED)
+          ap[j] = __fadd_rn(__fmul_rn(frac[__ldg(codes8 + b)], __ldg(scales + (b >> 8))),
+                            __ldg(absmax + (b >> 8)));
+        else
+          ap[j] = codes8 ? __fmul_rn(frac[__ldg(codes8 + b)], __ldg(scales + (b >> 8)))
+                         : __ldg(absmax + b);
       }
     }
 #pragma unroll
@@ -103,6 +107,40 @@ __global__ void __launch_bounds__(256) k_dequant(const uint8_t* __restrict__ pac
 
 using namespace aqnf4;
 
+namespace {
+
+aqnf4_status launch_dequant(const uint8_t* packed, const uint8_t* codes8, const float* scales,
+                            const float* absmax, int64_t n, int32_t out_dtype, void* out,
+                            bool centered, cudaStream_t stream) {
+  const Tables* tb = default_tables();
+  if (!tb) return AQNF4_ERR_CUDA;
+  DqParams p;
+  for (int i = 0; i < 16; ++i) p.level[i] = tb->level[i];
+  const int64_t nchunk = (n + 7) >> 3;
+  const int64_t groups = (nchunk + 32 * kChunksPerLane - 1) / (32 * kChunksPerLane);
+  const int sms = current_sm_count();
+  int64_t grid = static_cast<int64_t>(sms > 0 ? sms : 1) * 8;  // 8 warps per CTA
+  const int64_t need = (groups + 7) / 8;
+  if (grid > need) grid = need;
+  uint16_t* o = static_cast<uint16_t*>(out);
+  const unsigned g = static_cast<unsigned>(grid);
+  if (out_dtype == AQNF4_BF16) {
+    if (centered)
+      k_dequant<AQNF4_BF16, true><<<g, 256, 0, stream>>>(packed, codes8, scales, absmax, n, o, p);
+    else
+      k_dequant<AQNF4_BF16, false><<<g, 256, 0, stream>>>(packed, codes8, scales, absmax, n, o, p);
+  } else {
+    if (centered)
+      k_dequant<AQNF4_F16, true><<<g, 256, 0, stream>>>(packed, codes8, scales, absmax, n, o, p);
+    else
+      k_dequant<AQNF4_F16, false><<<g, 256, 0, stream>>>(packed, codes8, scales, absmax, n, o, p);
+  }
+  count_launches(1);
+  return cudaGetLastError() == cudaSuccess ? AQNF4_OK : AQNF4_ERR_CUDA;
+}
+
+}  // namespace
+
 extern "C" aqnf4_status aqnf4_dequantize(const uint8_t* packed, const uint8_t* codes8,
                                          const float* scales, const float* absmax, int64_t n,
                                          int32_t out_dtype, void* out, cudaStream_t stream) {
@@ -112,29 +150,17 @@ extern "C" aqnf4_status aqnf4_dequantize(const uint8_t* packed, const uint8_t* c
   if (!is_aligned(packed, 16) || !is_aligned(out, 16) || !is_aligned(scales, 4) ||
       !is_aligned(absmax, 4))
     return AQNF4_ERR_ALIGNMENT;
-  const Tables* tb = default_tables();
-  if (!tb) return AQNF4_ERR_CUDA;
-  DqParams p;
-  for (int i = 0; i < 16; ++i) p.level[i] = tb->level[i];
-  const int64_t nchunk = (n + 7) >> 3;
-  const int64_t groups = (nchunk + 32 * kChunksPerLane - 1) / (32 * kChunksPerLane);
-  const int sms = current_sm_count();
-  int64_t grid = static_cast<int64_t>(sms > 0 ? sms : 1) * 8;  // 8 warps per CTA
-  if (AQNF4_DQ_OCC_GRID) {
-    int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_dequant<AQNF4_BF16>, 256, 0) ==
-            cudaSuccess && occ > 0)
-      grid = static_cast<int64_t>(sms > 0 ? sms : 1) * occ;
-  }
-  const int64_t need = (groups + 7) / 8;
-  if (grid > need) grid = need;
-  uint16_t* o = static_cast<uint16_t*>(out);
-  if (out_dtype == AQNF4_BF16)
-    k_dequant<AQNF4_BF16><<<static_cast<unsigned>(grid), 256, 0, stream>>>(packed, codes8, scales,
-                                                                           absmax, n, o, p);
-  else
-    k_dequant<AQNF4_F16><<<static_cast<unsigned>(grid), 256, 0, stream>>>(packed, codes8, scales,
-                                                                          absmax, n, o, p);
-  count_launches(1);
-  return cudaGetLastError() == cudaSuccess ? AQNF4_OK : AQNF4_ERR_CUDA;
+  return launch_dequant(packed, codes8, scales, absmax, n, out_dtype, out, false, stream);
+}
+
+extern "C" aqnf4_status aqnf4_dequantize_centered(const uint8_t* packed, const uint8_t* codes8,
+                                                  const float* scales, const float* means,
+                                                  int64_t n, int32_t out_dtype, void* out,
+                                                  cudaStream_t stream) {
+  if (!packed || !codes8 || !scales || !means || !out || n < 1) return AQNF4_ERR_INVALID_ARG;
+  if (!valid_dtype(out_dtype)) return AQNF4_ERR_DTYPE;
+  if (!is_aligned(packed, 16) || !is_aligned(out, 16) || !is_aligned(scales, 4) ||
+      !is_aligned(means, 4))
+    return AQNF4_ERR_ALIGNMENT;
+  return launch_dequant(packed, codes8, scales, means, n, out_dtype, out, true, stream);
 }

@@ -46,6 +46,7 @@ namespace {
 constexpr int kBpt = 2;
 constexpr int kThreads = kDqBlock / kBpt;  // a CTA covers one tile (= one DQ block)
 constexpr int kWarps = kThreads / 32;
+static_assert(kWarps == 4, "the centred score's tree takes slot bits 5..6 from 4 warps");
 // chunk loop of the coding pass unrolled by 2: smaller code, slightly faster than full unroll
 constexpr int kP2Unroll = 2;
 constexpr int kCtasPerSm = 5;  // 44 KB of shared memory and <= 102 registers per thread, no spills
@@ -67,7 +68,8 @@ constexpr size_t kRedOff = kOutOff + kPackedTileBytes;
 constexpr size_t kRedBytes = 3 * kDqBlock * sizeof(float);
 constexpr size_t kMaxOff = kRedOff + kRedBytes;
 constexpr size_t kPreOff = kMaxOff + 16 * sizeof(float);  // per-warp max for a DQ score
-constexpr size_t kBarOff = kPreOff + 16 * sizeof(float);
+constexpr size_t kCenOff = kPreOff + 16 * sizeof(float);  // per-warp sums for a centred score
+constexpr size_t kBarOff = kCenOff + 2 * kWarps * sizeof(double);
 constexpr size_t kSmemBytes = kBarOff + 16;
 
 struct LayerRec {
@@ -152,10 +154,11 @@ __device__ __forceinline__ void issue_tile(const QParams& p, int64_t tile, uint8
 }
 
 // Generic per-element path for a block whose absmax lies outside [2^-40, 2^40] (zero,
-// subnormal, huge or not finite).  Re-reads the block (natural element order) from shared
-// memory, rewrites this thread's packed words and returns the normalised sums (err, w^2) --
-// scaled by a^2 later like the fast path's.  ar is the constant w_hat is rebuilt from: a,
-// or the double-quantized a' (at most ~2a, so the normalised terms stay small).
+// subnormal, huge or not finite), or whose rebuild constant does.  Re-reads the block
+// (natural element order) from shared memory, rewrites this thread's packed words and
+// returns the sums (err, w^2) normalised by sb = max(a, |ar|) -- scaled by sb^2 later.  ar
+// is the constant w_hat is rebuilt from: a, or a double-quantized constant; normalising by
+// the larger of the two keeps every term at most about 4 whatever ar is.
 template <int DT, bool SCORE>
 __device__ __noinline__ float2 block_generic(const uint8_t* my, float a, float ar,
                                              const QParams& p,
@@ -169,6 +172,18 @@ __device__ __noinline__ float2 block_generic(const uint8_t* my, float a, float a
     as = __fmul_rn(a, scale);
   }
   const float r = zero ? 0.0f : __frcp_rn(as);
+  // normalisation of the error terms: by sb = max(a, |ar|) (= a unless ar exceeds it)
+  const float sb = fmaxf(a, fabsf(ar));
+  float escale = scale, er = r;
+  if (sb != a) {
+    escale = 1.0f;
+    float sbs = sb;
+    if (sb < 0x1p-126f) {
+      escale = 0x1p64f;
+      sbs = __fmul_rn(sb, escale);
+    }
+    er = __frcp_rn(sbs);
+  }
   const uint16_t* x16 = reinterpret_cast<const uint16_t*>(my);
   float se = 0.0f, sw = 0.0f;
   for (int c = 0; c < 8; ++c) {
@@ -184,11 +199,12 @@ __device__ __noinline__ float2 block_generic(const uint8_t* my, float a, float a
         for (int j = 0; j < 15; ++j) code += (v > p.mid[j]) ? 1 : 0;
       }
       pk |= static_cast<uint32_t>(code) << ((i >> 1) * 8 + ((i & 1) ? 0 : 4));
-      if (SCORE && !zero) {
+      if (SCORE && !(zero && ar == 0.0f)) {
         const float wh = F::round_trip(__fmul_rn(p.level[code], ar));
-        const float d = __fmul_rn(__fsub_rn(__fmul_rn(x, scale), __fmul_rn(wh, scale)), r);
+        const float d = __fmul_rn(__fsub_rn(__fmul_rn(x, escale), __fmul_rn(wh, escale)), er);
+        const float ve = sb == a ? v : __fmul_rn(__fmul_rn(x, escale), er);
         se = __fmaf_rn(d, d, se);
-        sw = __fmaf_rn(v, v, sw);
+        sw = __fmaf_rn(ve, ve, sw);
       }
     }
     *reinterpret_cast<uint32_t*>(ost + c * 4) = pk;
@@ -209,6 +225,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   float* red = reinterpret_cast<float*>(smem + kRedOff);   // [3 = err, w2, scale][256]
   float* wmax = reinterpret_cast<float*>(smem + kMaxOff);  // [kWarps]
   uint32_t* wpre = reinterpret_cast<uint32_t*>(smem + kPreOff);  // [kWarps]
+  double* wcen = reinterpret_cast<double*>(smem + kCenOff);       // [2][kWarps]
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kBarOff);
   int* abort_flag = reinterpret_cast<int*>(smem + kBarOff + 8);
   const uint32_t bar_a = smem_addr(bar);
@@ -294,6 +311,51 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       const float s = __uint_as_float(sb);
 #pragma unroll
       for (int b = 0; b < kBpt; ++b) ar[b] = dq_constant(dq_code(a[b], s), s);
+    } else if (SCORE && (L.flags & AQNF4_SCORE_DQ_CENTERED)) {
+      // mean-centred DQ constants of this tile (one DQ block): the binary64 sum over the
+      // balanced tree of its 256 slots, slot t + 128 b held by thread t.  Slot bits 0..4
+      // are the lane (xor butterfly), bits 5..6 the warp, bit 7 the half b; each pair sum
+      // is the same in both partners since binary64 addition is commutative.  Slots past
+      // the layer's end hold the padding's absmax, +0.
+      double v0 = static_cast<double>(a[0]), v1 = static_cast<double>(a[1]);
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        v0 = __dadd_rn(v0, __shfl_xor_sync(kFull, v0, off));
+        v1 = __dadd_rn(v1, __shfl_xor_sync(kFull, v1, off));
+      }
+      if (lane == 0) {
+        wcen[warp] = v0;
+        wcen[kWarps + warp] = v1;
+      }
+      __syncthreads();
+      const double S = __dadd_rn(__dadd_rn(__dadd_rn(wcen[0], wcen[1]), __dadd_rn(wcen[2], wcen[3])),
+                                 __dadd_rn(__dadd_rn(wcen[4], wcen[5]), __dadd_rn(wcen[6], wcen[7])));
+      const float mu = __double2float_rn(__ddiv_rn(S, static_cast<double>(nblk)));
+      float c[kBpt];
+      uint32_t m = 0;
+#pragma unroll
+      for (int b = 0; b < kBpt; ++b) {
+        c[b] = __fsub_rn(a[b], mu);
+        // |c| >= 0 or NaN: as unsigned integers the patterns order like the values, NaN top
+        if (t + b * kThreads < nblk) m = max(m, __float_as_uint(fabsf(c[b])));
+      }
+      m = __reduce_max_sync(kFull, m);
+      if (lane == 0) wpre[warp] = m;
+      __syncthreads();
+      uint32_t hb = 0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) hb = max(hb, wpre[w]);
+      const float h = __uint_as_float(hb);
+      const bool finite = (fabsf(mu) <= FLT_MAX) && (h <= FLT_MAX);
+#pragma unroll
+      for (int b = 0; b < kBpt; ++b) {
+        int q = -128;  // a non-finite block stores code 0
+        if (finite) q = h == 0.0f ? 0 : __float2int_rn(__fmul_rn(__fdiv_rn(c[b], h), 127.0f));
+        ar[b] = __fadd_rn(__fmul_rn(__fdiv_rn(static_cast<float>(q), 127.0f), h), mu);
+        // a centred constant need not stay near a (a tile mixing tiny and huge blocks):
+        // the binary32 fast path's range argument needs |ar| <= 2^40 as well
+        if (!(fabsf(ar[b]) <= 0x1p40f)) fast[b] = false;
+      }
     }
 
     // ---- pass 2: codes, packing, error; the blocks' chains interleave (all lanes run this
@@ -368,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       float sum_scale = 1.0f;
       if (!fast[b]) {
         sums = block_generic<DT, SCORE>(stage + blk * 128, a[b], ar[b], p, ost + blk * 32);
-        sum_scale = a[b];
+        sum_scale = fmaxf(a[b], fabsf(ar[b]));  // block_generic's normalisation
       }
       if (SCORE) {
         r_err[blk] = sums.x;
@@ -532,7 +594,9 @@ void fill_tables(QParams& p, const Tables& tb) {
 }
 
 aqnf4_status check_layer(const aqnf4_layer& L) {
-  if (!L.w || L.numel < 1 || (L.flags & ~AQNF4_SCORE_DQ_ABSMAX) != 0) return AQNF4_ERR_INVALID_ARG;
+  const int32_t score_bits = AQNF4_SCORE_DQ_ABSMAX | AQNF4_SCORE_DQ_CENTERED;
+  if (!L.w || L.numel < 1 || (L.flags & ~score_bits) != 0 || L.flags == score_bits)
+    return AQNF4_ERR_INVALID_ARG;
   if (!valid_dtype(L.dtype)) return AQNF4_ERR_DTYPE;
   if (L.codes8 && !L.scales) return AQNF4_ERR_INVALID_ARG;
   if (!is_aligned(L.w, 16) || !is_aligned(L.packed, 16) || !is_aligned(L.absmax, 4) ||

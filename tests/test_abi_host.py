@@ -116,7 +116,7 @@ def test_argument_checks_return_before_any_launch(lib):
     one = (aqnf4.aqnf4_layer * 1)(layer())
     ws = V(0x100000)
     assert lib.aqnf4_layer_error(one, 0, ws, 4096, None, None, None, None, None) == aqnf4.AQNF4_ERR_INVALID_ARG
-    for flags in (2, 4, -1):  # only AQNF4_SCORE_DQ_ABSMAX is defined
+    for flags in (3, 4, -1):  # unknown bits, or both score flags at once
         bad = (aqnf4.aqnf4_layer * 1)(layer(flags=flags))
         assert lib.aqnf4_layer_error(bad, 1, ws, 4096, None, None, None, None, None) == \
             aqnf4.AQNF4_ERR_INVALID_ARG
@@ -158,6 +158,13 @@ def test_argument_checks_return_before_any_launch(lib):
     big = list(gemm)
     big[2] = 65535 * 256 + 1
     assert lib.aqnf4_nf4_linear(*big) == aqnf4.AQNF4_ERR_INVALID_ARG
+    # mean-centred DQ and its dequantization
+    assert lib.aqnf4_double_quant_centered(V(0x100), 0, V(0x200), V(0x300), V(0x400), None, None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert lib.aqnf4_double_quant_centered(V(0x100), 10, V(0x200), V(0x300), None, None, None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert lib.aqnf4_double_quant_centered(V(0x100), 10, V(0x200), V(0x300), V(0x402), None, None) == aqnf4.AQNF4_ERR_ALIGNMENT
+    assert lib.aqnf4_dequantize_centered(V(0x100), V(0x200), V(0x300), None, 64, 1, V(0x500), None) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert lib.aqnf4_dequantize_centered(V(0x100), V(0x200), V(0x300), V(0x400), 64, 7, V(0x500), None) == aqnf4.AQNF4_ERR_DTYPE
+    assert lib.aqnf4_dequantize_centered(V(0x108), V(0x200), V(0x300), V(0x400), 64, 1, V(0x500), None) == aqnf4.AQNF4_ERR_ALIGNMENT
     # division diagnostic
     assert lib.aqnf4_selftest_division(V(0x100), V(0x200), 0, V(0x300), None) == aqnf4.AQNF4_ERR_INVALID_ARG
     assert lib.aqnf4_selftest_division(None, V(0x200), 4, V(0x300), None) == aqnf4.AQNF4_ERR_INVALID_ARG

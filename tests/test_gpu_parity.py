@@ -241,6 +241,61 @@ def test_double_quant_nonfinite_flag(cuda):
     assert same_float_bits(scales.cpu().numpy(), osc)
 
 
+def test_double_quant_centered_matches_oracle(cuda):
+    """Mean-centred DQ (an option from outside the pages): codes, h and mean bit-exact on
+    ragged sizes, wide and narrow value ranges, a constant block, a zero block, subnormal
+    and huge constants mixed with ordinary ones."""
+    rng = np.random.default_rng(15)
+    cases = []
+    for nb in (1, 2, 255, 256, 257, 1000, 4096 + 3, 30000):
+        a = np.abs(rng.standard_normal(nb)).astype(np.float32) * 0.03
+        if nb > 600:
+            a[256:512] = np.float32(0.0125)   # a constant block: h = 0, codes 128
+            a[512:520] = 0.0                  # zeros inside a block
+        cases.append(a)
+    wide = np.abs(rng.standard_normal(2048)).astype(np.float32) * \
+        np.exp2(rng.integers(-30, 30, 2048)).astype(np.float32)
+    wide[:5] = [1e-40, 3e-39, 2.0 ** -140, 1e30, 0.0]  # subnormal, tiny and huge constants
+    cases.append(wide)
+    for a in cases:
+        codes8, scales, means = aqnf4.double_quant_centered(torch.from_numpy(a).to(cuda))
+        oc, osc, omu, _ = oracle.double_quant_centered(a)
+        assert np.array_equal(codes8.cpu().numpy(), oc), a.size
+        assert same_float_bits(scales.cpu().numpy(), osc), a.size
+        assert same_float_bits(means.cpu().numpy(), omu), a.size
+
+
+def test_double_quant_centered_nonfinite_flag(cuda):
+    a = np.full(600, 0.5, np.float32)
+    a[300] = np.nan
+    a[10] = np.inf
+    flag = torch.zeros(1, dtype=torch.int32, device=cuda)
+    nd = 3
+    codes8 = torch.empty(600, dtype=torch.uint8, device=cuda)
+    scales = torch.empty(nd, dtype=torch.float32, device=cuda)
+    means = torch.empty(nd, dtype=torch.float32, device=cuda)
+    aqnf4.aqnf4_double_quant_centered(torch.from_numpy(a).to(cuda), codes8, scales, means, flag)
+    assert flag.item() == aqnf4.AQNF4_ERR_NONFINITE
+    oc, osc, omu, onf = oracle.double_quant_centered(a)
+    assert onf
+    assert np.array_equal(codes8.cpu().numpy(), oc)
+    assert same_float_bits(scales.cpu().numpy(), osc)
+    assert same_float_bits(means.cpu().numpy(), omu)
+
+
+@pytest.mark.parametrize("out_dt", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("n", [1, 9, 64, 65, 16384 + 3, 200001])
+def test_dequantize_centered_matches_oracle(cuda, out_dt, n):
+    w = synth.random_bits_host(n, seed=n + 17, dtype=torch.bfloat16)
+    op, oa, _ = oracle.quantize(bits(w), oracle.BF16)
+    oc, osc, omu, _ = oracle.double_quant_centered(oa)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(cuda)
+    out = torch.empty(n, dtype=out_dt, device=cuda)
+    aqnf4.aqnf4_dequantize_centered(dev(op), dev(oc), dev(osc), dev(omu), n, out)
+    ref = oracle.dequantize_centered(op, n, DT[out_dt], oc, osc, omu)
+    assert np.array_equal(bits(out.cpu()), ref)
+
+
 @pytest.mark.parametrize("out_dt", [torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("n", [1, 2, 7, 8, 9, 63, 64, 65, 1023, 16384 + 3, 200001])
 def test_dequantize_matches_oracle(cuda, out_dt, n):
@@ -387,6 +442,45 @@ def test_dq_score_matches_oracle_and_keeps_the_storage(cuda):
         assert rel[i].item() == pytest.approx(orel, rel=RTOL), i
         for name in ("packed", "codes8", "scales"):  # the flag changes only the score
             assert torch.equal(getattr(dq_st[i], name), getattr(plain_st[i], name)), (i, name)
+
+
+def test_centered_dq_score_matches_oracle_and_keeps_the_storage(cuda):
+    """The score against mean-centred DQ constants (a format from outside the pages) within
+    1e-5 of the oracle's, on ragged layers with zero, tiny and huge blocks; the stored
+    outputs stay the plain format's."""
+    ws = _dq_case_layers()
+    dev = [w.to(cuda) for w in ws]
+    plain_st = [aqnf4.NF4Storage(w.numel(), cuda) for w in dev]
+    dq_st = [aqnf4.NF4Storage(w.numel(), cuda) for w in dev]
+    aqnf4.score_layers(dev, plain_st)
+    se, sw, rel = aqnf4.score_layers(dev, dq_st, dq_score="centered")
+    torch.cuda.synchronize()
+    for i, w in enumerate(ws):
+        ose, osw, orel = oracle.layer_error_dqc(bits(w), DT[w.dtype])
+        assert se[i].item() == pytest.approx(ose, rel=RTOL), i
+        assert sw[i].item() == pytest.approx(osw, rel=RTOL), i
+        assert rel[i].item() == pytest.approx(orel, rel=RTOL), i
+        for name in ("packed", "codes8", "scales"):
+            assert torch.equal(getattr(dq_st[i], name), getattr(plain_st[i], name)), (i, name)
+
+
+def test_three_scores_in_one_call(cuda):
+    """Flags are per layer: plain, DQ-absmax and centred scores mixed in one launch."""
+    ws = _dq_case_layers()
+    dev = [w.to(cuda) for w in ws]
+    modes = [0, aqnf4.AQNF4_SCORE_DQ_ABSMAX, aqnf4.AQNF4_SCORE_DQ_CENTERED]
+    refs = [oracle.layer_error, oracle.layer_error_dq, oracle.layer_error_dqc]
+    descs = aqnf4.make_layers([{"w": w, "flags": modes[i % 3]} for i, w in enumerate(dev)])
+    L = len(dev)
+    wsp = torch.empty(max(256, aqnf4.aqnf4_workspace_size(descs)), dtype=torch.uint8, device=cuda)
+    se = torch.empty(L, dtype=torch.float64, device=cuda)
+    rel = torch.empty(L, dtype=torch.float32, device=cuda)
+    aqnf4.aqnf4_layer_error(descs, wsp, se, None, rel)
+    torch.cuda.synchronize()
+    for i, w in enumerate(ws):
+        ose, _, orel = refs[i % 3](bits(w), DT[w.dtype])
+        assert se[i].item() == pytest.approx(ose, rel=RTOL), i
+        assert rel[i].item() == pytest.approx(orel, rel=RTOL), i
 
 
 def test_dq_and_plain_scores_in_one_call(cuda):
