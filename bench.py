@@ -366,6 +366,7 @@ def run_native(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": max(3, args.warmup), "ms_per_step": elapsed_ms / K, "higher_is_better": True,
         "scaling": "strong", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "layers_per_s": L * K / (elapsed_ms / 1e3),
         "config": {
             "workload": workload_desc(wl), "layers": L, "weight_bytes": total_weight_bytes,
             "budget_bytes": budget, "k_cap": wl.k_cap,
@@ -377,7 +378,13 @@ def run_native(args):
             "outputs": "packed NF4 + 8-bit DQ codes + fp32 DQ scales + per-layer scores",
         },
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic, "kernel": "k_quant_score",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "traffic_source": ("profiles/k_quant_score_7b.md: ncu dram__bytes_read.sum + "
+                                        "dram__bytes_write.sum of one full-size launch, taken on "
+                                        "kernel sources with the recorded sha256")
+                     if traffic is not None else
+                     "none: no ncu capture recorded for the current kernel sources",
+                     "kernel": "k_quant_score",
                      "peak_source": f"{peak_src} hbm_gbs", "alg_bytes_per_launch": my_alg,
                      "launch_ms": kern_avg_ms},
         "clocks": clocks.summary(),
@@ -439,8 +446,39 @@ def run_native(args):
         dist.barrier(device_ids=[local])
         dist.destroy_process_group()
     if rank == 0:
+        result["summary"] = compact_summary(result)  # last: a tail of the line keeps it
         print(json.dumps(result), flush=True)
     return 0
+
+
+def compact_summary(r):
+    """The line's figures in a few hundred bytes: the main kernel's roofline fraction and
+    layers/s, the other model shapes, the dequantize kernel (named shape and sweep points
+    with the same-traffic copy floor), the fused GEMM against dequantize + cuBLAS, and the
+    DQ-absmax score."""
+    def rnd(x, d=4):
+        return None if x is None else round(float(x), d)
+    s = {"frac": rnd(r["roofline"]["frac"]), "gbs": rnd(r["value"], 1),
+         "layers_per_s": rnd(r.get("layers_per_s"), 1)}
+    for name, w in (r.get("workloads") or {}).items():
+        s[name] = {"frac": rnd(w["roofline"]["frac"]), "gbs": rnd(w["value"], 1),
+                   "layers_per_s": rnd(w.get("layers_per_s"), 1)}
+    if "dequant" in r:
+        d = r["dequant"]
+        s["dequant"] = {"shape": d["shape"], "gbs": rnd(d["value"], 1),
+                        "frac": rnd(d["roofline"]["frac"])}
+    pts = {p["case"]: p for p in (r.get("dequant_sweep") or {}).get("points", [])}
+    for case in ("packed_8MB", "packed_16MB", "packed_1024MB"):
+        if case in pts:
+            s.setdefault("dequant", {})[case] = [rnd(pts[case]["frac"], 3),
+                                                 rnd(pts[case].get("copy_frac"), 3)]
+    if "nf4_linear" in r:
+        for k, v in r["nf4_linear"].items():
+            if k.startswith("tokens_"):
+                s[f"gemm_{k}"] = [rnd(v["value"], 1), rnd(v.get("dequant_then_cublas"), 1)]
+    if "dq_score" in r:
+        s["dq_score_frac"] = rnd(r["dq_score"]["roofline"]["frac"])
+    return s
 
 
 def measured_tensor_peak():
@@ -617,6 +655,7 @@ def bench_dq_score(weights, stor, wl, cost, budget, sel_plain, k_plain, dev, str
     kept = sorted(sel[:k].tolist())
     kept_plain = sorted(sel_plain[:k_plain].tolist())
     return {"value": wl.weight_bytes / (ms / 1e3) / 1e9, "unit": UNIT, "ms_per_step": ms,
+            "layers_per_s": len(weights) / (ms / 1e3),
             "steps": steps,
             "roofline": {"bound": "hbm", "achieved": alg / (kern_ms / 1e3) / 1e9, "peak": peak,
                          "unit": "GB/s", "frac": alg / (kern_ms / 1e3) / 1e9 / peak,
@@ -675,6 +714,7 @@ def bench_workload(name, dev, stream, peak, steps):
     dts = sorted({str(s.dtype).replace("torch.", "") for s in wl.layers})
     return {"workload": workload_desc(wl), "dtype_in": "/".join(dts), "steps": steps,
             "ms_per_step": ms, "value": wl.weight_bytes / (ms / 1e3) / 1e9, "unit": UNIT,
+            "layers_per_s": L / (ms / 1e3),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "kernel": "k_quant_score",
                          "launch_ms": kern_ms, "alg_bytes_per_launch": alg},
@@ -763,13 +803,33 @@ def bench_dequant_sweep(dev, stream, peak, reps=9):
         ms = sorted(times)[reps // 2]
         alg = dequant_alg_bytes(n)
         gbs = alg / (ms / 1e3) / 1e9
+        # the memory floor at this size: a device copy moving the same bytes (alg / 2 read,
+        # alg / 2 written), timed the same way from a flushed L2
+        src = torch.empty(alg // 2, dtype=torch.uint8, device=dev)
+        dst = torch.empty_like(src)
+        ctimes = []
+        for _ in range(reps):
+            with torch.cuda.stream(stream):
+                flush.fill_(1)
+                clean.sum()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            with torch.cuda.stream(stream):
+                dst.copy_(src)
+            b.record(stream)
+            b.synchronize()
+            ctimes.append(a.elapsed_time(b))
+        cms = sorted(ctimes)[reps // 2]
         points.append({"case": name, "packed_bytes": n // 2, "elements": n,
-                       "us": ms * 1e3, "value": gbs, "frac": gbs / peak})
-        del st, out
+                       "us": ms * 1e3, "value": gbs, "frac": gbs / peak,
+                       "copy_us": cms * 1e3, "copy_frac": alg / (cms / 1e3) / 1e9 / peak})
+        del st, out, src, dst
     torch.cuda.empty_cache()
     return {"unit": "GB/s", "peak": peak, "kernel": "k_dequant", "dtype_out": "bfloat16",
             "l2": "flushed before every launch (256 MB write, then 256 MB read); median of %d"
                   % reps,
+            "copy_reference": "copy_frac: a device copy of the same byte count (half read, "
+                              "half written), same flush and timing: the floor at that size",
             "points": points}
 
 

@@ -1,6 +1,7 @@
 """Host logic of bench.py that needs no GPU: the session command line, the algorithmic
 byte counts its rooflines divide by."""
 import importlib.util
+import json
 import os
 
 import pytest
@@ -54,3 +55,29 @@ def test_profile_commands_parse(bench, monkeypatch):
     for name, argv in cmds:
         monkeypatch.setattr("sys.argv", ["bench.py"] + argv)
         bench.parse_args()  # exits on an unknown or malformed argument
+
+
+def test_compact_summary_fits_the_line_tail(bench):
+    """The summary that ends the JSON line keeps every headline figure in well under the
+    1500 bytes of a line's tail."""
+    rf = {"frac": 0.61234567, "achieved": 4000.0}
+    wl = {"value": 3000.0, "layers_per_s": 40000.0, "roofline": rf}
+    r = {"value": 3100.0, "layers_per_s": 54000.0, "roofline": rf,
+         "workloads": {"14b": wl, "1.4b": wl},
+         "dequant": {"shape": "28672x8192", "value": 5600.0, "roofline": rf},
+         "dequant_sweep": {"points": [{"case": c, "frac": 0.5, "copy_frac": 0.6}
+                                      for c in ("packed_1MB", "packed_8MB", "packed_16MB",
+                                                "packed_1024MB")]},
+         "nf4_linear": {"unit": "TFLOP/s", "tokens_4096": {"value": 1000.0,
+                                                            "dequant_then_cublas": 1400.0},
+                        "tokens_128": {"value": 260.0, "dequant_then_cublas": 280.0}},
+         "dq_score": {"roofline": rf}}
+    s = bench.compact_summary(r)
+    r["summary"] = s
+    line = json.dumps(r)
+    assert line.endswith(json.dumps(s) + "}")
+    assert len(json.dumps(s)) < 1000
+    for key in ("frac", "layers_per_s", "14b", "1.4b", "dequant", "gemm_tokens_4096",
+                "gemm_tokens_128", "dq_score_frac"):
+        assert key in s
+    assert s["dequant"]["packed_8MB"] == [0.5, 0.6]
