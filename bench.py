@@ -411,6 +411,8 @@ def run_native(args):
         result["nf4_linear"] = bench_nf4_linear(dev, stream)
 
     if world == 1 and not args.no_dq_score:
+        result["dqc_score"] = bench_dq_score(weights, stor, wl, cost, budget, sel, k_sel, dev,
+                                             stream, peak, steps=min(K, 100), mode="centered")
         result["dq_score"] = bench_dq_score(weights, stor, wl, cost, budget, sel, k_sel, dev,
                                             stream, peak, steps=min(K, 100))
 
@@ -478,6 +480,8 @@ def compact_summary(r):
                 s[f"gemm_{k}"] = [rnd(v["value"], 1), rnd(v.get("dequant_then_cublas"), 1)]
     if "dq_score" in r:
         s["dq_score_frac"] = rnd(r["dq_score"]["roofline"]["frac"])
+    if "dqc_score" in r:
+        s["dqc_score_frac"] = rnd(r["dqc_score"]["roofline"]["frac"])
     return s
 
 
@@ -611,15 +615,18 @@ def bench_select_blocks(wl, se, sw, cost, budget, dev, stream, reps=200):
     return out
 
 
-def bench_dq_score(weights, stor, wl, cost, budget, sel_plain, k_plain, dev, stream, peak, steps):
+def bench_dq_score(weights, stor, wl, cost, budget, sel_plain, k_plain, dev, stream, peak, steps,
+                   mode="absmax"):
     """The same scoring step with every layer scored against its double-quantized constants
-    (AQNF4_SCORE_DQ_ABSMAX): GB/s of weights read, the fused kernel's roofline fraction, and
+    (mode "absmax": AQNF4_SCORE_DQ_ABSMAX; "centered": AQNF4_SCORE_DQ_CENTERED, the
+    mean-centred format): GB/s of weights read, the fused kernel's roofline fraction, and
     whether the kept set under the budget differs from the plain score's."""
     import torch
 
     from quantized_lora_setup_b200 import aqnf4
+    flag = {"absmax": aqnf4.AQNF4_SCORE_DQ_ABSMAX, "centered": aqnf4.AQNF4_SCORE_DQ_CENTERED}[mode]
     descs = aqnf4.make_layers([{"w": w, "packed": s.packed, "codes8": s.codes8,
-                                "scales": s.scales, "flags": aqnf4.AQNF4_SCORE_DQ_ABSMAX}
+                                "scales": s.scales, "flags": flag}
                                for w, s in zip(weights, stor)])
     L = len(weights)
     ws = torch.empty(max(256, aqnf4.aqnf4_workspace_size(descs)), dtype=torch.uint8, device=dev)
@@ -659,7 +666,9 @@ def bench_dq_score(weights, stor, wl, cost, budget, sel_plain, k_plain, dev, str
             "steps": steps,
             "roofline": {"bound": "hbm", "achieved": alg / (kern_ms / 1e3) / 1e9, "peak": peak,
                          "unit": "GB/s", "frac": alg / (kern_ms / 1e3) / 1e9 / peak,
-                         "kernel": "k_quant_score (AQNF4_SCORE_DQ_ABSMAX)"},
+                         "kernel": "k_quant_score (%s)" % ("AQNF4_SCORE_DQ_ABSMAX"
+                                                           if mode == "absmax" else
+                                                           "AQNF4_SCORE_DQ_CENTERED")},
             "selected": {"k": k, "of": L, "same_set_as_plain_score": kept == kept_plain}}
 
 

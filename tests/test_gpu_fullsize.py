@@ -136,17 +136,20 @@ def test_full_size_dequantize(cuda):
     assert 0.005 < float(err.sqrt()) < 0.15
 
 
-def test_full_model_dq_score_sampled_layers(cuda):
-    """The 7B-shaped model scored against its double-quantized constants, as bench.py's
-    dq_score line times it: sampled layers against the oracle within 1e-5."""
+@pytest.mark.parametrize("mode", ["absmax", "centered"])
+def test_full_model_dq_score_sampled_layers(cuda, mode):
+    """The 7B-shaped model scored against its double-quantized constants (plain 8-bit DQ, and
+    the mean-centred format), as bench.py's dq_score and dqc_score lines time it: sampled
+    layers against the oracle within 1e-5."""
     wl = synth.workload("7b")
     weights = [synth.layer_device(s, wl.seed, i, cuda) for i, s in enumerate(wl.layers)]
-    se, sw, rel = aqnf4.score_layers(weights, None, dq_score=True)
+    se, sw, rel = aqnf4.score_layers(weights, None, dq_score=mode)
     torch.cuda.synchronize()
     sample = _sample(wl)
     jobs = [(weights[i].cpu(), DT[wl.layers[i].dtype]) for i in sample]
+    ref = oracle.layer_error_dq if mode == "absmax" else oracle.layer_error_dqc
     with ThreadPoolExecutor(max_workers=len(jobs)) as ex:
-        results = list(ex.map(lambda a: oracle.layer_error_dq(synth.bits_u16(a[0]), a[1]), jobs))
+        results = list(ex.map(lambda a: ref(synth.bits_u16(a[0]), a[1]), jobs))
     for i, (ose, osw, orel) in zip(sample, results):
         assert se[i].item() == pytest.approx(ose, rel=RTOL), i
         assert sw[i].item() == pytest.approx(osw, rel=RTOL), i
