@@ -365,15 +365,31 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
 
 // Split K: y = sum over z of the binary32 partials ws[z], added in split order (the result
 // does not depend on scheduling), converted to y's format.  If the GEMM reported a timeout in
-// the caller's flag word, some partials were never written: y is left alone.
+// the caller's flag word, some partials were never written: y is left alone.  When M N is a
+// multiple of 4 every split's partials stay 16-byte aligned, and each thread sums four
+// consecutive outputs with 16-byte loads; otherwise it sums one output at a time.
 template <int DT>
 __global__ void __launch_bounds__(256) k_splitk_reduce(const float* __restrict__ ws, int splits,
                                                        int64_t mn, void* y, int out_f32,
                                                        const int32_t* flag) {
   using F = Fmt<DT>;
   if (flag && *reinterpret_cast<const volatile int32_t*>(flag) == AQNF4_ERR_TIMEOUT) return;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < mn;
-       i += static_cast<int64_t>(gridDim.x) * 256) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * 256;
+  const int64_t nvec = (mn & 3) == 0 ? mn >> 2 : 0;
+  for (int64_t v = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; v < nvec; v += stride) {
+    float4 acc = __ldcs(reinterpret_cast<const float4*>(ws) + v);
+    for (int z = 1; z < splits; ++z) {
+      const float4 u = __ldcs(reinterpret_cast<const float4*>(ws + z * mn) + v);
+      acc = make_float4(__fadd_rn(acc.x, u.x), __fadd_rn(acc.y, u.y), __fadd_rn(acc.z, u.z),
+                        __fadd_rn(acc.w, u.w));
+    }
+    if (out_f32)
+      reinterpret_cast<float4*>(y)[v] = acc;
+    else
+      reinterpret_cast<uint2*>(y)[v] = make_uint2(F::pack_rn(acc.x, acc.y), F::pack_rn(acc.z, acc.w));
+  }
+  for (int64_t i = 4 * nvec + static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < mn;
+       i += stride) {
     float acc = __ldcs(ws + i);
     for (int z = 1; z < splits; ++z) acc = __fadd_rn(acc, __ldcs(ws + z * mn + i));
     if (out_f32)
@@ -427,7 +443,7 @@ cudaError_t launch_gemm(const CUtensorMap& map, const GParams& p, cudaStream_t s
   count_launches(1);
   if (p.splits > 1) {
     const int64_t mn = p.M * p.N;
-    int64_t blocks = (mn + 255) / 256;
+    int64_t blocks = ((mn & 3) == 0 ? mn / 4 + 255 : mn + 255) / 256;
     const int64_t cap = static_cast<int64_t>(current_sm_count() > 0 ? current_sm_count() : 148) * 8;
     if (blocks > cap) blocks = cap;
     k_splitk_reduce<DT><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p.ws, p.splits, mn,

@@ -63,9 +63,11 @@ def test_nf4_linear_matches_oracle(cuda, dt, M, N, K):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
-@pytest.mark.parametrize("M,N,K", [(128, 11008, 4096), (16, 1024, 2048), (300, 512, 8192)])
+@pytest.mark.parametrize("M,N,K", [(128, 11008, 4096), (16, 1024, 2048), (300, 512, 8192),
+                                   (7, 1023, 2048)])
 def test_nf4_linear_split_k_matches_oracle(cuda, dt, M, N, K):
-    """Few output tiles: K is split over several CTAs whose partials are added in order."""
+    """Few output tiles: K is split over several CTAs whose partials are added in order (four
+    outputs per thread when M N is a multiple of 4, one at a time otherwise: 7 x 1023)."""
     assert aqnf4.aqnf4_nf4_linear_workspace_size(M, N, K) > 0
     x, packed, codes8, scales = _case(M, N, K, dt, seed=K + M)
     ref, rabs = oracle.nf4_linear(synth.bits_u16(x).reshape(M, K), DT[dt], packed, codes8,
@@ -75,6 +77,9 @@ def test_nf4_linear_split_k_matches_oracle(cuda, dt, M, N, K):
     y2 = _run(cuda, x, packed, codes8, scales, N, torch.float32)
     assert np.all(np.abs(y1 - ref) <= bound)
     assert np.array_equal(y1, y2)  # the partial sums are added in a fixed order
+    y16 = _run(cuda, x, packed, codes8, scales, N, dt)
+    ulp = 2.0 ** -8 if dt == torch.bfloat16 else 2.0 ** -11
+    assert np.all(np.abs(y16 - ref) <= bound + ulp * (np.abs(ref) + bound) + 6e-8)
 
 
 @pytest.mark.gpu
