@@ -532,11 +532,9 @@ def bench_nf4_linear(dev, stream, reps=20, shapes=((4096, 11008, 4096), (128, 11
         g.manual_seed(M)
         x = torch.randn((M, K), generator=g, device=dev).to(torch.bfloat16)
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        ws = torch.empty(max(16, aqnf4.aqnf4_nf4_linear_workspace_size(M, N, K)),
-                         dtype=torch.uint8, device=dev)
 
         def fused():
-            aqnf4.aqnf4_nf4_linear(x, st.packed, st.codes8, st.scales, N, y, None, stream, ws)
+            aqnf4.aqnf4_nf4_linear(x, st.packed, st.codes8, st.scales, N, y, None, stream)
 
         def unfused():
             aqnf4.aqnf4_dequantize(st.packed, st.codes8, st.scales, None, N * K, wd, stream)
@@ -557,7 +555,7 @@ def bench_nf4_linear(dev, stream, reps=20, shapes=((4096, 11008, 4096), (128, 11
             res[name] = 2.0 * M * N * K / (ms / 1e3) / 1e12
         out[f"tokens_{M}"] = {
             "value": res["fused"], "ms": 2.0 * M * N * K / res["fused"] / 1e9,
-            "split_k": aqnf4.aqnf4_nf4_linear_workspace_size(M, N, K) > 0,
+            "split_k": aqnf4.aqnf4_nf4_linear_splits(M, N, K),
             "roofline": {"bound": "tensor", "achieved": res["fused"], "peak": peak,
                          "unit": "TFLOP/s", "frac": res["fused"] / peak,
                          "kernel": "k_nf4_gemm"},

@@ -227,25 +227,24 @@ AQNF4_API aqnf4_status aqnf4_layer_error_noalloc(const aqnf4_layer* layers, int3
    16-byte aligned), codes8 (device, N*K/64 bytes), scales (device, ceil(N*K/16384) floats):
    the layer's storage as aqnf4_layer_error writes it; y (device, M x N, row-major,
    16-byte aligned): float when out_f32 != 0, else dtype.  K must be a positive multiple of 64, so that each row of
-   the layer is whole NF4 blocks.  workspace (optional, device, 16-byte aligned) of ws_bytes:
-   when the output has too few 256 x 256 tiles to fill the GPU, K is split over several thread
-   blocks whose binary32 partial sums go there and are then added in a fixed order; with at
-   least aqnf4_nf4_linear_workspace_size(M, N, K) bytes the split is used, otherwise the call
-   runs unsplit (still correct).  dev_flag (optional, device int32) receives
-   AQNF4_ERR_TIMEOUT if a bounded wait inside the kernel gave up; y is then not written by
-   the split-K sum and its tiles are not meaningful (without a dev_flag a timeout goes
-   unreported and y is undefined).
+   the layer is whole NF4 blocks.  When the output has too few 256 x 256 tiles to fill the
+   GPU, K is split over aqnf4_nf4_linear_splits(M, N, K) thread blocks that form one cluster
+   per tile and add their binary32 partial sums on chip, in split order (the result does not
+   depend on scheduling, and no workspace is needed).  dev_flag (optional, device int32)
+   receives AQNF4_ERR_TIMEOUT if a bounded wait inside the kernel gave up; the tiles that
+   wait belonged to are then not written (without a dev_flag a timeout goes unreported and y
+   is undefined).
    Errors: INVALID_ARG (NULL pointer, M < 1, N < 1, K not a positive multiple of 64, sizes
    above 2^31, M above 65535 * 256 = 16776960 rows), DTYPE, ALIGNMENT, CUDA. */
 AQNF4_API aqnf4_status aqnf4_nf4_linear(const void* x, int32_t dtype, int64_t M, int64_t K,
                                         const uint8_t* packed, const uint8_t* codes8,
                                         const float* scales, int64_t N, void* y,
-                                        int32_t out_f32, void* workspace, size_t ws_bytes,
-                                        int32_t* dev_flag, cudaStream_t stream);
+                                        int32_t out_f32, int32_t* dev_flag,
+                                        cudaStream_t stream);
 
-/* Workspace bytes aqnf4_nf4_linear uses to split K for this shape on the current device (0:
-   it does not split).  Host only. */
-AQNF4_API size_t aqnf4_nf4_linear_workspace_size(int64_t M, int64_t N, int64_t K);
+/* How many thread blocks aqnf4_nf4_linear splits K over for this shape on the current device
+   (1: no split; at most 8; 0: invalid shape).  Host only. */
+AQNF4_API int32_t aqnf4_nf4_linear_splits(int64_t M, int64_t N, int64_t K);
 
 /* Top-K under a byte budget (arxivdaily 2608.23816, "English abstract": the highest-error
    layers stay in 16 bits while a byte budget allows; "AQLoRA: ...", "Technical Details":

@@ -101,11 +101,10 @@ def library() -> ctypes.CDLL:
     lib.aqnf4_selftest_wait_timeout.restype = st
     lib.aqnf4_selftest_division.argtypes = [P, P, i64, P, P]
     lib.aqnf4_selftest_division.restype = st
-    lib.aqnf4_nf4_linear.argtypes = [P, i32, i64, i64, P, P, P, i64, P, i32, P,
-                                     ctypes.c_size_t, P, P]
+    lib.aqnf4_nf4_linear.argtypes = [P, i32, i64, i64, P, P, P, i64, P, i32, P, P]
     lib.aqnf4_nf4_linear.restype = st
-    lib.aqnf4_nf4_linear_workspace_size.argtypes = [i64, i64, i64]
-    lib.aqnf4_nf4_linear_workspace_size.restype = ctypes.c_size_t
+    lib.aqnf4_nf4_linear_splits.argtypes = [i64, i64, i64]
+    lib.aqnf4_nf4_linear_splits.restype = i32
     lib.aqnf4_select_blocks.argtypes = [P, P, P, P, i32, i32, i64, i32, P, P, P, P, P]
     lib.aqnf4_select_blocks.restype = st
     lib.aqnf4_slot_tables.argtypes = [P, P, P]
@@ -341,10 +340,9 @@ def aqnf4_selftest_division(a: torch.Tensor, s: torch.Tensor, out: torch.Tensor,
 
 def aqnf4_nf4_linear(x: torch.Tensor, packed: torch.Tensor, codes8: torch.Tensor,
                      scales: torch.Tensor, N: int, y: torch.Tensor,
-                     dev_flag: Optional[torch.Tensor] = None, stream=None,
-                     workspace: Optional[torch.Tensor] = None) -> None:
+                     dev_flag: Optional[torch.Tensor] = None, stream=None) -> None:
     """y (M x N) = x (M x K) w_hat^T for the N x K layer stored as packed + codes8 + scales;
-    y may be float32 or x's dtype.  workspace: see aqnf4_nf4_linear_workspace_size."""
+    y may be float32 or x's dtype."""
     if x.dim() != 2:
         raise ValueError("x must be M x K")
     M, K = x.shape
@@ -357,17 +355,14 @@ def aqnf4_nf4_linear(x: torch.Tensor, packed: torch.Tensor, codes8: torch.Tensor
     _req(codes8, "codes8", (torch.uint8,), nb)
     _req(scales, "scales", (torch.float32,), nsc)
     _req(y, "y", None, M * N)
-    _req(workspace, "workspace", None, optional=True)
     _req(dev_flag, "dev_flag", (torch.int32,), 1, optional=True)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(library().aqnf4_nf4_linear(_ptr(x), dtype_code(x.dtype), M, K, _ptr(packed),
                                       _ptr(codes8), _ptr(scales), N, _ptr(y), out_f32,
-                                      _ptr(workspace), ws_bytes, _ptr(dev_flag),
-                                      _stream(stream)), "aqnf4_nf4_linear")
+                                      _ptr(dev_flag), _stream(stream)), "aqnf4_nf4_linear")
 
 
-def aqnf4_nf4_linear_workspace_size(M: int, N: int, K: int) -> int:
-    return int(library().aqnf4_nf4_linear_workspace_size(M, N, K))
+def aqnf4_nf4_linear_splits(M: int, N: int, K: int) -> int:
+    return int(library().aqnf4_nf4_linear_splits(M, N, K))
 
 
 def aqnf4_select_blocks(sq_err: torch.Tensor, sq_w: torch.Tensor, block_of: torch.Tensor,

@@ -50,6 +50,11 @@ constexpr int kBarBase = kRingB + kStagesB * kTileBytesB;   // after the rings
 constexpr int kFracOff = kBarBase + 256;                     // fl(c / 255) for c = 0..255
 constexpr int kGSmemBytes = kFracOff + 1024 + 1024;         // + alignment slack
 constexpr uint32_t kTmemCols = 512;  // two f32 accumulators of 256 columns: all of TMEM
+// split K: the splits of one output tile form a thread-block cluster (portable size <= 8);
+// each stages a 128 x 256 binary32 accumulator in its (then idle) rings for the others
+constexpr int kMaxSplits = 8;
+constexpr int kStageBytes = 128 * kBN * 4;
+static_assert(kStageBytes <= kBarBase, "the staged accumulator fits in the rings");
 static_assert(kDeqWarps * 16 == kBN, "two dequantizing threads per row of the w_hat tile");
 
 struct GParams {
@@ -59,9 +64,9 @@ struct GParams {
   void* y;
   int64_t M, N, K;
   int32_t out_f32;
-  int32_t splits;  // K is split over gridDim.z CTAs; > 1: partial sums go to ws
-  float* ws;       // [splits][M][N] binary32 partial sums (splits > 1)
+  int32_t splits;     // K is split over the gridDim.z CTAs of one cluster (<= kMaxSplits)
   int32_t* flag;
+  int32_t a_rows;     // rows of x one copy brings: 128 when M <= 128 (the rest unused)
   float level[16];
 };
 
@@ -138,6 +143,34 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Thread-block cluster: a barrier over all threads of the cluster (release / acquire: the
+// shared-memory writes before it are visible to every CTA of the cluster after it), the
+// address of the same shared-memory location in CTA `rank`, and loads from there.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ float4 ld_cluster_v4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant__ CUtensorMap tmap_x,
                                                            const __grid_constant__ GParams p) {
@@ -153,6 +186,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
   uint64_t* accum = empty_b + kStagesB;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accum + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* fail_word = const_cast<int*>(abort_flag) + 1;  // split K: read by the cluster's CTAs
   float* frac = reinterpret_cast<float*>(smem + kFracOff);
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -201,7 +235,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
           *abort_flag = 1;
           break;
         }
-        mbar_arrive_expect_tx(smem_addr(full_a + s), kTileBytesA);
+        mbar_arrive_expect_tx(smem_addr(full_a + s), static_cast<uint32_t>(p.a_rows) * kBK * 2);
         tma_load_2d(smem_addr(smem + s * kTileBytesA), &tmap_x,
                     static_cast<int>((kt0 + i) * kBK), static_cast<int>(m0),
                     smem_addr(full_a + s));
@@ -304,9 +338,8 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
   const bool ready = warp < kDeqWarps ? mbar_wait_bounded(smem_addr(accum), 0) : true;
   const int failed = __syncthreads_or(!ready || *abort_flag);
   tc_fence_after();
-  if (failed) {
-    if (t == 0 && p.flag) *p.flag = AQNF4_ERR_TIMEOUT;
-  } else if (warp < kDeqWarps) {
+  if (failed && t == 0 && p.flag) *p.flag = AQNF4_ERR_TIMEOUT;
+  if (p.splits == 1 && !failed && warp < kDeqWarps) {
     // warp w: TMEM lanes 32 (w mod 4).. ; accumulator (w / 8) holds rows 128 (w / 8).. of the
     // tile; columns 128 ((w / 4) mod 2)..
     const int q = warp & 3, acc = warp >> 3, chalf = (warp >> 2) & 1;
@@ -319,9 +352,8 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
       const int64_t col = n0 + cbase;
       if (m < p.M && col < p.N) {
         const bool whole = col + 32 <= p.N;
-        if (p.splits > 1 || p.out_f32) {
-          float* dst = p.splits > 1 ? p.ws + (blockIdx.z * p.M + m) * p.N + col
-                                    : static_cast<float*>(p.y) + m * p.N + col;
+        if (p.out_f32) {
+          float* dst = static_cast<float*>(p.y) + m * p.N + col;
           if (whole && (p.N & 3) == 0) {
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
@@ -346,6 +378,88 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
       }
     }
   }
+  if (p.splits > 1) {
+    // Split K over the cluster's CTAs (cluster rank = blockIdx.z = split).  For each
+    // 128-row accumulator: every CTA stages its binary32 partial in its own rings (row-major,
+    // 16-byte chunk j of row r at position j ^ (r mod 8), so that neither the staging stores
+    // nor the reads below conflict on banks); after a cluster barrier, CTA z adds, for rows
+    // [z rows / S, (z + 1) rows / S), the S partials in split order (the bits do not depend
+    // on scheduling) through distributed shared memory and stores y; a second barrier keeps
+    // every CTA's rings alive until the others have read them.  Every thread of the cluster
+    // takes the same barriers; if any CTA of the cluster timed out, no CTA writes y.
+    const int S = p.splits, z = static_cast<int>(blockIdx.z);
+    if (t == 0) *fail_word = failed;
+    const int cols = static_cast<int>(p.N - n0 < kBN ? p.N - n0 : kBN);
+    const bool vec = (p.N & 3) == 0;
+    const uint32_t stage = smem_addr(smem);
+    int any_failed = 0;
+    for (int hh = 0; hh < (lower_half ? 2 : 1); ++hh) {
+      const int64_t r0 = m0 + 128 * hh;  // first row of y in this accumulator
+      const int rows = static_cast<int>(p.M - r0 < 128 ? p.M - r0 : 128);
+      if (!failed && warp < kDeqWarps && 32 * (warp & 3) < rows) {
+        // warp w: TMEM lanes 32 (w mod 4).. = rows; columns 64 (w / 4)..
+        const int q = warp & 3, cq = warp >> 2;
+        const int r = 32 * q + lane;
+        uint8_t* row = smem + r * (kBN * 4);
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          float v[32];
+          const int cbase = 64 * cq + 32 * c;
+          tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + kBN * hh + cbase, v);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int j = cbase / 4 + i;
+            *reinterpret_cast<float4*>(row + ((j ^ (r & 7)) << 4)) =
+                make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          }
+        }
+      }
+      cluster_sync();
+      if (hh == 0)
+        for (int s2 = 0; s2 < S; ++s2)
+          any_failed |= ld_cluster_s32(cluster_map(smem_addr(fail_word), static_cast<uint32_t>(s2)));
+      if (!any_failed) {
+        const int lo = rows * z / S, hi = rows * (z + 1) / S;
+        uint32_t peer[kMaxSplits];
+#pragma unroll
+        for (int s2 = 0; s2 < kMaxSplits; ++s2)
+          peer[s2] = s2 < S ? cluster_map(stage, static_cast<uint32_t>(s2)) : 0u;
+        const int nchunk = (cols + 3) >> 2;
+        for (int e = t; e < (hi - lo) * nchunk; e += kGThreads) {
+          const int r = lo + e / nchunk, j = e % nchunk;
+          const uint32_t off = static_cast<uint32_t>(r * (kBN * 4) + ((j ^ (r & 7)) << 4));
+          float4 u[kMaxSplits];
+#pragma unroll
+          for (int s2 = 0; s2 < kMaxSplits; ++s2)
+            if (s2 < S) u[s2] = ld_cluster_v4(peer[s2] + off);
+          float4 acc = u[0];
+#pragma unroll
+          for (int s2 = 1; s2 < kMaxSplits; ++s2)
+            if (s2 < S)
+              acc = make_float4(__fadd_rn(acc.x, u[s2].x), __fadd_rn(acc.y, u[s2].y),
+                                __fadd_rn(acc.z, u[s2].z), __fadd_rn(acc.w, u[s2].w));
+          const int64_t i = (r0 + r) * p.N + n0 + 4 * j;
+          if (vec) {  // N, hence cols, a multiple of 4: whole 16- (8-) byte stores
+            if (p.out_f32)
+              *reinterpret_cast<float4*>(static_cast<float*>(p.y) + i) = acc;
+            else
+              *reinterpret_cast<uint2*>(static_cast<uint16_t*>(p.y) + i) =
+                  make_uint2(F::pack_rn(acc.x, acc.y), F::pack_rn(acc.z, acc.w));
+          } else {
+            const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+            for (int k = 0; k < 4 && 4 * j + k < cols; ++k) {
+              if (p.out_f32)
+                static_cast<float*>(p.y)[i + k] = a4[k];
+              else
+                static_cast<uint16_t*>(p.y)[i + k] =
+                    static_cast<uint16_t>(F::pack_rn(a4[k], 0.0f) & 0xffffu);
+            }
+          }
+        }
+      }
+      cluster_sync();
+    }
+  }
   if (warp == kProducerWarp && lane == 0 && failed) {
     // let every copy issued land before the shared memory goes away: tile s last received
     // step s + kStagesA * ((issued - 1 - s) / kStagesA)
@@ -363,51 +477,15 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
   }
 }
 
-// Split K: y = sum over z of the binary32 partials ws[z], added in split order (the result
-// does not depend on scheduling), converted to y's format.  If the GEMM reported a timeout in
-// the caller's flag word, some partials were never written: y is left alone.  When M N is a
-// multiple of 4 every split's partials stay 16-byte aligned, and each thread sums four
-// consecutive outputs with 16-byte loads; otherwise it sums one output at a time.
-template <int DT>
-__global__ void __launch_bounds__(256) k_splitk_reduce(const float* __restrict__ ws, int splits,
-                                                       int64_t mn, void* y, int out_f32,
-                                                       const int32_t* flag) {
-  using F = Fmt<DT>;
-  if (flag && *reinterpret_cast<const volatile int32_t*>(flag) == AQNF4_ERR_TIMEOUT) return;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * 256;
-  const int64_t nvec = (mn & 3) == 0 ? mn >> 2 : 0;
-  for (int64_t v = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; v < nvec; v += stride) {
-    float4 acc = __ldcs(reinterpret_cast<const float4*>(ws) + v);
-    for (int z = 1; z < splits; ++z) {
-      const float4 u = __ldcs(reinterpret_cast<const float4*>(ws + z * mn) + v);
-      acc = make_float4(__fadd_rn(acc.x, u.x), __fadd_rn(acc.y, u.y), __fadd_rn(acc.z, u.z),
-                        __fadd_rn(acc.w, u.w));
-    }
-    if (out_f32)
-      reinterpret_cast<float4*>(y)[v] = acc;
-    else
-      reinterpret_cast<uint2*>(y)[v] = make_uint2(F::pack_rn(acc.x, acc.y), F::pack_rn(acc.z, acc.w));
-  }
-  for (int64_t i = 4 * nvec + static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < mn;
-       i += stride) {
-    float acc = __ldcs(ws + i);
-    for (int z = 1; z < splits; ++z) acc = __fadd_rn(acc, __ldcs(ws + z * mn + i));
-    if (out_f32)
-      static_cast<float*>(y)[i] = acc;
-    else
-      static_cast<uint16_t*>(y)[i] = static_cast<uint16_t>(F::pack_rn(acc, 0.0f) & 0xffffu);
-  }
-}
-
 // Splits of K for a grid too small to fill the GPU: enough CTAs for one wave, at least 8
-// steps of 64 per split, at most 16 splits.
+// steps of 64 per split, at most kMaxSplits (one cluster per output tile).
 int choose_splits(int64_t M, int64_t N, int64_t K) {
   const int sms = current_sm_count() > 0 ? current_sm_count() : 148;
   const int64_t tiles = ((N + kBN - 1) / kBN) * ((M + kBM - 1) / kBM);
   if (tiles >= sms) return 1;
   int64_t s = sms / tiles;
   s = s < (K / kBK) / 8 ? s : (K / kBK) / 8;
-  s = s < 16 ? s : 16;
+  s = s < kMaxSplits ? s : kMaxSplits;
   return s >= 2 ? static_cast<int>(s) : 1;
 }
 
@@ -431,26 +509,60 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
+// Whether a cluster of `splits` CTAs of this kernel can be resident at once (one CTA per SM:
+// it needs that many SMs of one GPC); asked once per device, kernel and size.
+bool cluster_fits(const void* kern, int splits) {
+  static std::mutex mu;
+  static int known[16][2][kMaxSplits + 1];  // 0 unknown, 1 fits, 2 does not
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return false;
+  const int which = kern == reinterpret_cast<const void*>(k_nf4_gemm<AQNF4_BF16>) ? 0 : 1;
+  std::lock_guard<std::mutex> lock(mu);
+  int& k = known[dev][which][splits];
+  if (k == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, 1, static_cast<unsigned>(splits));
+    cfg.blockDim = dim3(kGThreads);
+    cfg.dynamicSmemBytes = kGSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = static_cast<unsigned>(splits);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    k = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) == cudaSuccess && clusters >= 1 ? 1 : 2;
+    cudaGetLastError();  // a refused query leaves no error behind
+  }
+  return k == 1;
+}
+
 template <int DT>
 cudaError_t launch_gemm(const CUtensorMap& map, const GParams& p, cudaStream_t stream) {
   auto kern = k_nf4_gemm<DT>;
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmemBytes);
   if (err != cudaSuccess) return err;
+  GParams q = p;
+  if (q.splits > 1 && !cluster_fits(reinterpret_cast<const void*>(kern), q.splits)) q.splits = 1;
   const dim3 grid(static_cast<unsigned>((p.N + kBN - 1) / kBN),
-                  static_cast<unsigned>((p.M + kBM - 1) / kBM), static_cast<unsigned>(p.splits));
-  kern<<<grid, kGThreads, kGSmemBytes, stream>>>(map, p);
+                  static_cast<unsigned>((p.M + kBM - 1) / kBM), static_cast<unsigned>(q.splits));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kGThreads);
+  cfg.dynamicSmemBytes = kGSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;  // the splits of a tile: one cluster
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = static_cast<unsigned>(q.splits);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  err = cudaLaunchKernelEx(&cfg, kern, map, q);
   count_launches(1);
-  if (p.splits > 1) {
-    const int64_t mn = p.M * p.N;
-    int64_t blocks = ((mn & 3) == 0 ? mn / 4 + 255 : mn + 255) / 256;
-    const int64_t cap = static_cast<int64_t>(current_sm_count() > 0 ? current_sm_count() : 148) * 8;
-    if (blocks > cap) blocks = cap;
-    k_splitk_reduce<DT><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p.ws, p.splits, mn,
-                                                                           p.y, p.out_f32, p.flag);
-    count_launches(1);
-  }
-  return cudaGetLastError();
+  return err;
 }
 
 }  // namespace
@@ -458,17 +570,16 @@ cudaError_t launch_gemm(const CUtensorMap& map, const GParams& p, cudaStream_t s
 
 using namespace aqnf4;
 
-extern "C" size_t aqnf4_nf4_linear_workspace_size(int64_t M, int64_t N, int64_t K) {
+extern "C" int32_t aqnf4_nf4_linear_splits(int64_t M, int64_t N, int64_t K) {
   if (M < 1 || N < 1 || K < kBK || K % kBK != 0) return 0;
-  const int s = choose_splits(M, N, K);
-  return s > 1 ? static_cast<size_t>(s) * static_cast<size_t>(M) * static_cast<size_t>(N) * 4 : 0;
+  return choose_splits(M, N, K);
 }
 
 extern "C" aqnf4_status aqnf4_nf4_linear(const void* x, int32_t dtype, int64_t M, int64_t K,
                                          const uint8_t* packed, const uint8_t* codes8,
                                          const float* scales, int64_t N, void* y,
-                                         int32_t out_f32, void* workspace, size_t ws_bytes,
-                                         int32_t* dev_flag, cudaStream_t stream) {
+                                         int32_t out_f32, int32_t* dev_flag,
+                                         cudaStream_t stream) {
   if (!x || !packed || !codes8 || !scales || !y || M < 1 || N < 1 || K < kBK || K % kBK != 0)
     return AQNF4_ERR_INVALID_ARG;
   if (M > (int64_t(1) << 31) - kBM || N > (int64_t(1) << 31) - kBN || K > (int64_t(1) << 31))
@@ -485,7 +596,8 @@ extern "C" aqnf4_status aqnf4_nf4_linear(const void* x, int32_t dtype, int64_t M
   CUtensorMap map;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-  const cuuint32_t box[2] = {kBK, kBM};
+  // a layer product of at most 128 tokens copies only the x rows it has
+  const cuuint32_t box[2] = {kBK, static_cast<cuuint32_t>(M <= 128 ? 128 : kBM)};
   const cuuint32_t estr[2] = {1, 1};
   if (encode(&map,
              dtype == AQNF4_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -504,11 +616,8 @@ extern "C" aqnf4_status aqnf4_nf4_linear(const void* x, int32_t dtype, int64_t M
   p.K = K;
   p.out_f32 = out_f32 ? 1 : 0;
   p.splits = choose_splits(M, N, K);
-  p.ws = static_cast<float*>(workspace);
-  if (p.splits > 1 && (!workspace || !is_aligned(workspace, 16) ||
-                       ws_bytes < static_cast<size_t>(p.splits) * M * N * 4))
-    p.splits = 1;  // no room for the partial sums: one CTA per output tile
   p.flag = dev_flag;
+  p.a_rows = M <= 128 ? 128 : kBM;
   for (int i = 0; i < 16; ++i) p.level[i] = tb->level[i];
   const cudaError_t err = dtype == AQNF4_BF16 ? launch_gemm<AQNF4_BF16>(map, p, stream)
                                               : launch_gemm<AQNF4_F16>(map, p, stream);

@@ -110,11 +110,9 @@ class SplitModel:
         M = x.shape[0]
         y = torch.empty((M, N), dtype=out_dtype if out_dtype == torch.float32 else x.dtype,
                         device=x.device)
-        nbytes = aqnf4.aqnf4_nf4_linear_workspace_size(M, N, K)
-        ws = torch.empty(nbytes, dtype=torch.uint8, device=x.device) if nbytes else None
         st = L.nf4
         aqnf4.aqnf4_nf4_linear(x.contiguous(), st.packed, st.codes8, st.scales, N, y,
-                               stream=stream, workspace=ws)
+                               stream=stream)
         return y.to(out_dtype)
 
     def memory_report(self) -> dict:

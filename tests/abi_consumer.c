@@ -28,8 +28,9 @@ int main(void) {
          (int)aqnf4_dequantize(NULL, NULL, NULL, NULL, 64, AQNF4_BF16, NULL, NULL));
   printf("nf4_linear_bad_k %d\n",
          (int)aqnf4_nf4_linear((const void*)16, AQNF4_BF16, 4, 96, (const uint8_t*)16,
-                               (const uint8_t*)16, (const float*)16, 8, (void*)16, 1, NULL, 0,
-                               NULL, NULL));
+                               (const uint8_t*)16, (const float*)16, 8, (void*)16, 1, NULL,
+                               NULL));
+  printf("nf4_linear_splits_bad_k %d\n", (int)aqnf4_nf4_linear_splits(4, 8, 96));
   printf("launches %llu\n", (unsigned long long)(aqnf4_launch_count() - before));
   printf("status %s\n", aqnf4_status_string(AQNF4_ERR_ALIGNMENT));
   return 0;

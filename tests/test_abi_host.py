@@ -154,7 +154,7 @@ def test_argument_checks_return_before_any_launch(lib):
     assert lib.aqnf4_selftest_wait_timeout(1000, V(0x102), None, None) == aqnf4.AQNF4_ERR_ALIGNMENT
     # fused GEMM: row tiles beyond the grid's y limit are rejected up front
     gemm = [V(0x100), aqnf4.AQNF4_BF16, 65535 * 256, 64, V(0x200), V(0x300), V(0x400), 256,
-            V(0x500), 0, None, 0, None, None]
+            V(0x500), 0, None, None]
     big = list(gemm)
     big[2] = 65535 * 256 + 1
     assert lib.aqnf4_nf4_linear(*big) == aqnf4.AQNF4_ERR_INVALID_ARG
@@ -261,5 +261,6 @@ def test_header_is_plain_c_and_links(lib, tmp_path):
     assert int(kv["layer_error_null_w"]) == aqnf4.AQNF4_ERR_INVALID_ARG
     assert int(kv["dequantize_null"]) == aqnf4.AQNF4_ERR_INVALID_ARG
     assert int(kv["nf4_linear_bad_k"]) == aqnf4.AQNF4_ERR_INVALID_ARG
+    assert int(kv["nf4_linear_splits_bad_k"]) == 0
     assert int(kv["launches"]) == 0
     assert out.splitlines()[-1] == "status " + aqnf4.status_string(aqnf4.AQNF4_ERR_ALIGNMENT)

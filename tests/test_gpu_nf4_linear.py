@@ -25,17 +25,13 @@ def _case(M, N, K, dt, seed):
     return x, packed, codes8, scales
 
 
-def _run(cuda, x, packed, codes8, scales, N, out_dtype, split=True):
+def _run(cuda, x, packed, codes8, scales, N, out_dtype):
     M, K = x.shape
     y = torch.full((M, N), float("nan"), dtype=out_dtype, device=cuda)
     flag = torch.zeros(1, dtype=torch.int32, device=cuda)
-    ws = None
-    if split:
-        nbytes = aqnf4.aqnf4_nf4_linear_workspace_size(M, N, K)
-        ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=cuda)
     aqnf4.aqnf4_nf4_linear(x.to(cuda), torch.from_numpy(packed).to(cuda),
                            torch.from_numpy(codes8).to(cuda), torch.from_numpy(scales).to(cuda),
-                           N, y, flag, workspace=ws)
+                           N, y, flag)
     torch.cuda.synchronize()
     assert flag.item() == 0
     return y.double().cpu().numpy()
@@ -56,19 +52,22 @@ def test_nf4_linear_matches_oracle(cuda, dt, M, N, K):
     y16 = _run(cuda, x, packed, codes8, scales, N, dt)
     ulp = 2.0 ** -8 if dt == torch.bfloat16 else 2.0 ** -11
     assert np.all(np.abs(y16 - ref) <= bound + ulp * (np.abs(ref) + bound) + 6e-8)
-    # without a workspace the call runs unsplit: same bound
-    y32u = _run(cuda, x, packed, codes8, scales, N, torch.float32, split=False)
-    assert np.all(np.abs(y32u - ref) <= bound)
 
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
-@pytest.mark.parametrize("M,N,K", [(128, 11008, 4096), (16, 1024, 2048), (300, 512, 8192),
-                                   (7, 1023, 2048)])
-def test_nf4_linear_split_k_matches_oracle(cuda, dt, M, N, K):
-    """Few output tiles: K is split over several CTAs whose partials are added in order (four
-    outputs per thread when M N is a multiple of 4, one at a time otherwise: 7 x 1023)."""
-    assert aqnf4.aqnf4_nf4_linear_workspace_size(M, N, K) > 0
+@pytest.mark.parametrize("M,N,K,S", [(128, 11008, 4096, 3), (16, 1024, 2048, 4),
+                                     (300, 512, 8192, 8), (7, 1023, 2048, 4),
+                                     (300, 6400, 1024, 2), (128, 5376, 3584, 7),
+                                     (200, 10240, 2048, 3)])
+def test_nf4_linear_split_k_matches_oracle(cuda, dt, M, N, K, S):
+    """Few output tiles: K is split over the S CTAs of a cluster, which add their partials
+    on chip in split order (16-byte stores when N is a multiple of 4, one output at a time
+    otherwise: 7 x 1023; two row tiles, the second ragged: 300 x ...; both 128-row halves of
+    one tile: 200 x 10240)."""
+    if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+        assert aqnf4.aqnf4_nf4_linear_splits(M, N, K) == S
+    assert aqnf4.aqnf4_nf4_linear_splits(M, N, K) > 1
     x, packed, codes8, scales = _case(M, N, K, dt, seed=K + M)
     ref, rabs = oracle.nf4_linear(synth.bits_u16(x).reshape(M, K), DT[dt], packed, codes8,
                                   scales, N, DT[dt])
@@ -107,7 +106,7 @@ def test_nf4_linear_rejects_bad_shapes():
     V = __import__("ctypes").c_void_p
     before = lib.aqnf4_launch_count()
     args = [V(0x1000), aqnf4.AQNF4_BF16, 4, 64, V(0x2000), V(0x3000), V(0x4000), 8, V(0x5000),
-            1, None, 0, None, None]
+            1, None, None]
     for i, bad in ((3, 0), (3, 96), (3, 63), (2, 0), (7, 0), (0, None), (8, None)):
         a = list(args)
         a[i] = bad
@@ -123,19 +122,24 @@ def test_nf4_linear_rejects_bad_shapes():
         a[8], a[9] = V(y), out_f32
         assert lib.aqnf4_nf4_linear(*a) == aqnf4.AQNF4_ERR_ALIGNMENT, (out_f32, y)
     assert lib.aqnf4_launch_count() == before
-    assert aqnf4.aqnf4_nf4_linear_workspace_size(4, 8, 96) == 0
+    assert aqnf4.aqnf4_nf4_linear_splits(4, 8, 96) == 0
 
 
-def test_split_k_workspace_sizes():
+def test_split_k_counts():
     """The split rule on a 148-SM part (what the library assumes without a device):
-    enough splits for one wave, at least 8 steps of 64 each, none when the tiles fill it."""
+    enough splits for one wave, at least 8 steps of 64 each, at most 8 (one cluster), none
+    when the tiles fill it."""
     if torch.cuda.is_available() and torch.cuda.get_device_properties(0).multi_processor_count != 148:
-        pytest.skip("sizes below are for 148 SMs")
+        pytest.skip("counts below are for 148 SMs")
     # 11008 x 4096 layer, 128 tokens: 43 output tiles -> 148 // 43 = 3 splits
-    assert aqnf4.aqnf4_nf4_linear_workspace_size(128, 11008, 4096) == 3 * 128 * 11008 * 4
+    assert aqnf4.aqnf4_nf4_linear_splits(128, 11008, 4096) == 3
     # 16 tokens, 1024 outputs, K 2048: 4 tiles -> 37, capped by 32 steps / 8 = 4
-    assert aqnf4.aqnf4_nf4_linear_workspace_size(16, 1024, 2048) == 4 * 16 * 1024 * 4
+    assert aqnf4.aqnf4_nf4_linear_splits(16, 1024, 2048) == 4
+    # 4 tiles, K 8192: 37, capped at 8 CTAs per cluster
+    assert aqnf4.aqnf4_nf4_linear_splits(300, 512, 8192) == 8
     # K = 512: 8 steps cannot be split into two halves of >= 8 steps
-    assert aqnf4.aqnf4_nf4_linear_workspace_size(16, 1024, 512) == 0
+    assert aqnf4.aqnf4_nf4_linear_splits(16, 1024, 512) == 1
     # 4096 tokens x 11008: 16 x 43 = 688 tiles fill the GPU: no split
-    assert aqnf4.aqnf4_nf4_linear_workspace_size(4096, 11008, 4096) == 0
+    assert aqnf4.aqnf4_nf4_linear_splits(4096, 11008, 4096) == 1
+    # not a valid shape
+    assert aqnf4.aqnf4_nf4_linear_splits(16, 1024, 100) == 0
