@@ -24,6 +24,9 @@
 //     the stage when they finish;
 //   - warps 0-15 then read the accumulators with tcgen05.ld (warp w: TMEM lanes 32(w mod 4)..,
 //     accumulator w / 8, columns 128 ((w / 4) mod 2)..) and store y.
+// When the output has too few tiles to fill the GPU, K is split over up to 8 CTAs that form
+// one thread-block cluster per tile; they add their partial sums through distributed shared
+// memory instead of a trip through HBM and a second kernel.
 // Every wait is bounded: a wait that gives up records AQNF4_ERR_TIMEOUT and makes every role
 // stop; copies in flight are allowed to land and the TMEM is always freed before exit.
 #include <cuda.h>
