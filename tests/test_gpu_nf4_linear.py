@@ -41,8 +41,11 @@ def _run(cuda, x, packed, codes8, scales, N, out_dtype):
 @pytest.mark.parametrize("dt", [torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("M,N,K", [(128, 128, 64), (1, 1, 64), (200, 300, 256),
                                    (256, 384, 4096), (130, 129, 192), (64, 100, 128),
-                                   (70, 260, 320)])
+                                   (70, 260, 320), (600, 300, 256), (520, 1000, 512),
+                                   (1024, 512, 960)])
 def test_nf4_linear_matches_oracle(cuda, dt, M, N, K):
+    """Shapes with one CTA per tile (several row tiles, an odd count: 600 and 520 rows) and
+    with split K."""
     x, packed, codes8, scales = _case(M, N, K, dt, seed=M + N + K)
     ref, rabs = oracle.nf4_linear(synth.bits_u16(x).reshape(M, K), DT[dt], packed, codes8,
                                   scales, N, DT[dt])
@@ -79,6 +82,27 @@ def test_nf4_linear_split_k_matches_oracle(cuda, dt, M, N, K, S):
     y16 = _run(cuda, x, packed, codes8, scales, N, dt)
     ulp = 2.0 ** -8 if dt == torch.bfloat16 else 2.0 ** -11
     assert np.all(np.abs(y16 - ref) <= bound + ulp * (np.abs(ref) + bound) + 6e-8)
+
+
+@pytest.mark.gpu
+def test_nf4_linear_full_mlp_shape_sampled_rows(cuda):
+    """The 7B MLP up-projection at 4096 tokens (11008 x 4096, bf16), as the bench times it:
+    rows of y from several row tiles and both 128-row halves of a tile, against the
+    oracle's product of those rows of x."""
+    M, N, K = 4096, 11008, 4096
+    x, packed, codes8, scales = _case(M, N, K, torch.bfloat16, seed=11)
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device=cuda)
+    flag = torch.zeros(1, dtype=torch.int32, device=cuda)
+    aqnf4.aqnf4_nf4_linear(x.to(cuda), torch.from_numpy(packed).to(cuda),
+                           torch.from_numpy(codes8).to(cuda), torch.from_numpy(scales).to(cuda),
+                           N, y, flag)
+    torch.cuda.synchronize()
+    assert flag.item() == 0
+    rows = np.array([0, 127, 128, 255, 256, 511, 1100, 2047, 2048, 3071, 4000, 4095])
+    ref, rabs = oracle.nf4_linear(synth.bits_u16(x[rows]).reshape(len(rows), K), oracle.BF16,
+                                  packed, codes8, scales, N, oracle.BF16)
+    got = y[torch.from_numpy(rows).to(cuda)].double().cpu().numpy()
+    assert np.all(np.abs(got - ref) <= K * 2.0 ** -23 * rabs + 1e-30)
 
 
 @pytest.mark.gpu
