@@ -464,6 +464,28 @@ def test_centered_dq_score_matches_oracle_and_keeps_the_storage(cuda):
             assert torch.equal(getattr(dq_st[i], name), getattr(plain_st[i], name)), (i, name)
 
 
+@pytest.mark.parametrize("extreme", ["smallest", "largest"])
+def test_centered_dq_score_h_at_either_extreme(cuda, extreme):
+    """h = max |a - mu| comes from the tile's smallest constant (255 blocks near 1, one zero
+    block: mu near 1) or from its largest (255 blocks near 1, one block of 1000)."""
+    rng = np.random.default_rng(41 if extreme == "smallest" else 42)
+    w = rng.uniform(-1.0, 1.0, size=(256, 64)).astype(np.float32)
+    w[:, 0] = 1.0  # every block's absmax is 1 ...
+    if extreme == "smallest":
+        w[77] = 0.0  # ... but one zero block
+    else:
+        w[77] *= 1000.0  # ... but one huge block
+    for dt in (torch.bfloat16, torch.float16):
+        x = torch.from_numpy(w.reshape(-1)).to(dt)
+        st = [aqnf4.NF4Storage(x.numel(), cuda)]
+        se, sw, rel = aqnf4.score_layers([x.to(cuda)], st, dq_score="centered")
+        torch.cuda.synchronize()
+        ose, osw, orel = oracle.layer_error_dqc(bits(x), DT[dt])
+        assert se[0].item() == pytest.approx(ose, rel=RTOL)
+        assert sw[0].item() == pytest.approx(osw, rel=RTOL)
+        assert rel[0].item() == pytest.approx(orel, rel=RTOL)
+
+
 def test_three_scores_in_one_call(cuda):
     """Flags are per layer: plain, DQ-absmax and centred scores mixed in one launch."""
     ws = _dq_case_layers()
