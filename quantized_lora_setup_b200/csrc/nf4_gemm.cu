@@ -26,7 +26,11 @@
 //     accumulator w / 8, columns 128 ((w / 4) mod 2)..) and store y.
 // When the output has too few tiles to fill the GPU, K is split over up to 8 CTAs that form
 // one thread-block cluster per tile; they add their partial sums through distributed shared
-// memory instead of a trip through HBM and a second kernel.
+// memory instead of a trip through HBM and a second kernel.  With two or more row tiles and
+// no split, two row tiles run on a CTA pair with two-CTA MMAs (tcgen05.mma.cta_group::2,
+// M = 256 of which 128 rows from each CTA, N = 256 of which each CTA holds and dequantizes
+// 128 w_hat rows): each CTA rebuilds half the w_hat tile, and the tensor cores read a
+// w_hat row from shared memory once per 512 rows of x instead of once per 128.
 // Every wait is bounded: a wait that gives up records AQNF4_ERR_TIMEOUT and makes every role
 // stop; copies in flight are allowed to land and the TMEM is always freed before exit.
 #include <cuda.h>
@@ -85,11 +89,12 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 }
 
 // Instruction descriptor: f32 accumulator, both operands DT (f16 = 0, bf16 = 1), K-major,
-// N = 256, M = 128 (one of the two row halves of the tile).
-template <int DT>
+// N = 256, M = 128 (one of the two row halves of the tile; a CTA pair's MMA: M = 256, 128
+// rows from each CTA).
+template <int DT, int M = 128>
 __host__ __device__ constexpr uint32_t idesc() {
   return (1u << 4) | (static_cast<uint32_t>(DT) << 7) | (static_cast<uint32_t>(DT) << 10) |
-         (static_cast<uint32_t>(kBN >> 3) << 17) | (static_cast<uint32_t>(128 >> 4) << 24);
+         (static_cast<uint32_t>(kBN >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
@@ -174,7 +179,45 @@ __device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
   return v;
 }
 
-template <int DT>
+// ---- CTA pair (two row tiles of y over one w_hat tile, one 1 x 2 x 1 cluster): the even
+// CTA (the leader) issues tcgen05.mma.cta_group::2 with M = 256 (128 rows of x from each
+// CTA) and N = 256, where each CTA holds 128 of the 256 w_hat rows; each CTA's TMEM receives
+// its own rows.  Both CTAs' x copies and dequantizing warps complete on the leader's
+// barriers; the leader's commits arrive on both CTAs' barriers.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x,
+                                                 int y, uint32_t leader_bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(map), "r"(x), "r"(y), "r"(leader_bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_f16_pair(uint32_t tmem, uint64_t da, uint64_t db,
+                                              uint32_t id, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+      "l"(da), "l"(db), "r"(id), "r"(accumulate)
+      : "memory");
+}
+
+// arrives on the barrier at this offset in both CTAs of the pair once the MMAs have finished
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
+  const uint16_t mask = 3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+      "[%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+
+// arrival on a barrier of another CTA of the cluster
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
+template <int DT, bool PAIR>
 __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant__ CUtensorMap tmap_x,
                                                            const __grid_constant__ GParams p) {
   using F = Fmt<DT>;
@@ -194,13 +237,25 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
 
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   if (t < 256) frac[t] = __fdiv_rn(static_cast<float>(t), 255.0f);  // correctly rounded
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * kBN;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kBM;
+  // tiles: column tile on grid x and row tile on y.  A pair's two CTAs are neighbours along
+  // grid x (the cluster's x, as a two-CTA MMA needs): cluster k = blockIdx.x / 2 takes column
+  // tile k mod (column tiles) of row tiles 2 (k / column tiles) + {0, 1}, so the clusters
+  // resident at once share their rows of x through L2, as the unpaired grid order does.
+  const int64_t col_tiles = (p.N + kBN - 1) / kBN;
+  const int64_t pair_k = static_cast<int64_t>(blockIdx.x >> 1);
+  const int64_t n0 = (PAIR ? pair_k % col_tiles : static_cast<int64_t>(blockIdx.x)) * kBN;
+  const int64_t m0 =
+      (PAIR ? 2 * (pair_k / col_tiles) + (blockIdx.x & 1) : static_cast<int64_t>(blockIdx.y)) *
+      kBM;
   const int64_t kb = p.K / kBK;  // NF4 blocks per row of w = k steps
   // this CTA's steps [kt0, kt1): split z of p.splits (the pipeline counts i = kt - kt0)
   const int64_t kt0 = kb * blockIdx.z / p.splits, kt1 = kb * (blockIdx.z + 1) / p.splits;
   const int64_t nk = kt1 - kt0;
   const bool lower_half = m0 + 128 < p.M;  // the tile's second 128 rows hold any of x
+  // CTA pair: rank q = blockIdx.x mod 2 (a 2 x 1 x 1 cluster); the leader (q = 0) issues the
+  // MMAs.  Its lower_half covers the partner's too (the partner's rows lie further down).
+  const uint32_t q_rank = PAIR ? (blockIdx.x & 1u) : 0u;
+  const bool mma_cta = !PAIR || q_rank == 0;
 
   if (t == 0) {
     for (int s = 0; s < kStagesA; ++s) {
@@ -208,19 +263,32 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
       mbar_init(smem_addr(empty_a + s), 1);
     }
     for (int s = 0; s < kStagesB; ++s) {
-      mbar_init(smem_addr(full_b + s), 32 * kDeqWarps);
+      // pair: one arrival per dequantizing warp of either CTA, on the leader's barrier
+      mbar_init(smem_addr(full_b + s), PAIR ? 2 * kDeqWarps : 32 * kDeqWarps);
       mbar_init(smem_addr(empty_b + s), 1);
     }
     mbar_init(smem_addr(accum), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
+  if (PAIR) {
+    __syncthreads();
+    cluster_sync();  // both CTAs' barriers exist before either arrives on the other's
+  }
   if (warp == kMmaWarp) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_addr(tmem_holder)),
-                 "r"(kTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if (PAIR) {  // the same warp of both CTAs allocates the pair's TMEM together
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_addr(tmem_holder)),
+                   "r"(kTmemCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_addr(tmem_holder)),
+                   "r"(kTmemCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -234,23 +302,37 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
       for (int64_t i = 0; i < nk && !*abort_flag; ++i) {
         const int s = static_cast<int>(i % kStagesA);
         const uint32_t use = static_cast<uint32_t>(i / kStagesA);
-        if (i >= kStagesA && !mbar_wait_bounded(smem_addr(empty_a + s), (use - 1) & 1)) {
+        if (i >= kStagesA &&
+            !(PAIR ? mbar_wait_bounded(smem_addr(empty_a + s), (use - 1) & 1)
+                   : mbar_wait_bounded(smem_addr(empty_a + s), (use - 1) & 1))) {
           *abort_flag = 1;
           break;
         }
-        mbar_arrive_expect_tx(smem_addr(full_a + s), static_cast<uint32_t>(p.a_rows) * kBK * 2);
-        tma_load_2d(smem_addr(smem + s * kTileBytesA), &tmap_x,
-                    static_cast<int>((kt0 + i) * kBK), static_cast<int>(m0),
-                    smem_addr(full_a + s));
+        if (PAIR) {  // both CTAs' copies complete on the leader's barrier
+          if (q_rank == 0) mbar_arrive_expect_tx(smem_addr(full_a + s), 2u * kTileBytesA);
+          tma_load_2d_pair(smem_addr(smem + s * kTileBytesA), &tmap_x,
+                           static_cast<int>((kt0 + i) * kBK), static_cast<int>(m0),
+                           cluster_map(smem_addr(full_a + s), 0u));
+        } else {
+          mbar_arrive_expect_tx(smem_addr(full_a + s), static_cast<uint32_t>(p.a_rows) * kBK * 2);
+          tma_load_2d(smem_addr(smem + s * kTileBytesA), &tmap_x,
+                      static_cast<int>((kt0 + i) * kBK), static_cast<int>(m0),
+                      smem_addr(full_a + s));
+        }
         issued = i + 1;
       }
     }
   } else if (warp == kMmaWarp) {
-    if (lane == 0) {
+    if (lane == 0 && mma_cta) {
       for (int64_t i = 0; i < nk && !*abort_flag; ++i) {
         const int sa = static_cast<int>(i % kStagesA), sb = static_cast<int>(i % kStagesB);
-        if (!mbar_wait_bounded(smem_addr(full_a + sa), static_cast<uint32_t>(i / kStagesA) & 1) ||
-            !mbar_wait_bounded(smem_addr(full_b + sb), static_cast<uint32_t>(i / kStagesB) & 1)) {
+        const uint32_t pa = static_cast<uint32_t>(i / kStagesA) & 1;
+        const uint32_t pb = static_cast<uint32_t>(i / kStagesB) & 1;
+        const bool ok = PAIR ? mbar_wait_bounded(smem_addr(full_a + sa), pa) &&
+                                   mbar_wait_bounded(smem_addr(full_b + sb), pb)
+                             : mbar_wait_bounded(smem_addr(full_a + sa), pa) &&
+                                   mbar_wait_bounded(smem_addr(full_b + sb), pb);
+        if (!ok) {
           *abort_flag = 1;
           break;
         }
@@ -260,40 +342,70 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
 #pragma unroll
         for (int j = 0; j < kBK / 16; ++j) {  // K = 16 per MMA: 32 bytes along the swizzled row
           // rows 0..127 of x into columns 0..255 of TMEM, rows 128..255 into 256..511; both
-          // use the same dequantized w_hat tile
-          umma_f16(tmem, sw128_desc(a0 + 32 * j), sw128_desc(b0 + 32 * j), idesc<DT>(),
-                   (i > 0 || j > 0) ? 1u : 0u);
-          if (lower_half)  // uniform: skipped when those 128 rows lie past M
-            umma_f16(tmem + kBN, sw128_desc(a0 + 128 * 128 + 32 * j), sw128_desc(b0 + 32 * j),
-                     idesc<DT>(), (i > 0 || j > 0) ? 1u : 0u);
+          // use the same dequantized w_hat tile (pair: the same rows of both CTAs' x, and
+          // the w_hat rows 0..127 held by the leader and 128..255 by the partner)
+          const uint32_t acc = (i > 0 || j > 0) ? 1u : 0u;
+          if (PAIR)
+            umma_f16_pair(tmem, sw128_desc(a0 + 32 * j), sw128_desc(b0 + 32 * j),
+                          idesc<DT, 256>(), acc);
+          else
+            umma_f16(tmem, sw128_desc(a0 + 32 * j), sw128_desc(b0 + 32 * j), idesc<DT>(), acc);
+          if (lower_half) {  // uniform: skipped when those 128 rows lie past M
+            if (PAIR)
+              umma_f16_pair(tmem + kBN, sw128_desc(a0 + 128 * 128 + 32 * j),
+                            sw128_desc(b0 + 32 * j), idesc<DT, 256>(), acc);
+            else
+              umma_f16(tmem + kBN, sw128_desc(a0 + 128 * 128 + 32 * j), sw128_desc(b0 + 32 * j),
+                       idesc<DT>(), acc);
+          }
         }
-        umma_commit(smem_addr(empty_a + sa));  // each arrives once the MMAs above have finished
-        umma_commit(smem_addr(empty_b + sb));
+        // each arrives once the MMAs above have finished (pair: in both CTAs)
+        if (PAIR) {
+          umma_commit_pair(smem_addr(empty_a + sa));
+          umma_commit_pair(smem_addr(empty_b + sb));
+        } else {
+          umma_commit(smem_addr(empty_a + sa));
+          umma_commit(smem_addr(empty_b + sb));
+        }
       }
-      umma_commit(smem_addr(accum));  // arrives once every MMA issued above has finished
+      // arrives once every MMA issued above has finished
+      if (PAIR)
+        umma_commit_pair(smem_addr(accum));
+      else
+        umma_commit(smem_addr(accum));
     }
   } else {
     // ---- dequantizing warps: threads 2r and 2r + 1 own the two halves of row n0 + r of the
-    // w_hat tile.  Step i's 16 bytes of packed codes, 8-bit constant and DQ scale are loaded
-    // from global memory while steps i - 3 .. i - 1 are worked on; the loop is unrolled by
-    // kStagesB (= 3), so step i + u always uses w_hat tile u and register set u.
+    // w_hat tile (pair: CTA q holds rows n0 + 128 q + r, r < 128, at tile row r; threads
+    // 4r .. 4r + 3 own its four quarters).  Step i's packed codes (16 or 8 bytes), 8-bit
+    // constant and DQ scale are loaded from global memory while steps i - 3 .. i - 1 are
+    // worked on; the loop is unrolled by kStagesB (= 3), so step i + u always uses w_hat tile
+    // u and register set u.
+    constexpr int kWords = PAIR ? 2 : 4;  // 32-bit words of packed codes per thread and step
     const float tab_level = p.level[lane & 15];  // lanes 16..31 mirror 0..15
-    const int r = t >> 1, hf = t & 1;
-    const int64_t n = n0 + r;
+    const int r = PAIR ? t >> 2 : t >> 1;
+    const int part = PAIR ? (t & 3) : (t & 1);
+    const int64_t n = n0 + 128 * static_cast<int64_t>(q_rank) + r;
     const bool row_ok = n < p.N;
-    const uint8_t* prow = p.packed + n * (p.K / 2) + hf * 16;
+    const uint8_t* prow = p.packed + n * (p.K / 2) + part * (4 * kWords);
     auto fetch = [&](int64_t kt, uint4& pk, uint32_t& c, float& s8) {
       if (row_ok && kt < kt1) {
         const int64_t b = n * kb + kt;
-        pk = __ldg(reinterpret_cast<const uint4*>(prow + kt * (kBK / 2)));
+        if (PAIR) {
+          const uint2 v = __ldg(reinterpret_cast<const uint2*>(prow + kt * (kBK / 2)));
+          pk = make_uint4(v.x, v.y, 0u, 0u);
+        } else {
+          pk = __ldg(reinterpret_cast<const uint4*>(prow + kt * (kBK / 2)));
+        }
         c = __ldg(p.codes8 + b);
         s8 = __ldg(p.scales + (b >> 8));
       }
     };
     // one step into w_hat tile u; false when the pipeline has been aborted
     auto dequant = [&](int64_t i, int u, const uint4& pk, uint32_t c8, float sc) -> bool {
-      bool ok = i < kStagesB ||
-                mbar_wait_bounded(smem_addr(empty_b + u), static_cast<uint32_t>(i / kStagesB - 1) & 1);
+      const uint32_t par = static_cast<uint32_t>(i / kStagesB - 1) & 1;
+      bool ok = i < kStagesB || (PAIR ? mbar_wait_bounded(smem_addr(empty_b + u), par)
+                                      : mbar_wait_bounded(smem_addr(empty_b + u), par));
       if (!ok) *abort_flag = 1;
       if (__any_sync(kFull, *abort_flag != 0)) return false;  // warp-uniform (shuffles below)
       // a zero constant (also for rows past N) gives 0
@@ -302,7 +414,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
       const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
       uint8_t* rowb = smem + kRingB + u * kTileBytesB + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
+      for (int jj = 0; jj < kWords; ++jj) {
         const uint32_t w = words[jj];
         uint32_t o[4];
 #pragma unroll
@@ -313,11 +425,21 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
           const f32x2 v = pmul_rn(pair(q0, q1), a2);
           o[h] = F::pack_rn(pair_lo(v), pair_hi(v));
         }
-        const int j = 4 * hf + jj;  // 16-byte chunk of the 128-byte row
+        const int j = kWords * part + jj;  // 16-byte chunk of the 128-byte row
         *reinterpret_cast<uint4*>(rowb + ((j ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
       }
       fence_proxy_async_smem();  // the tensor cores read this tile through the async proxy
-      mbar_arrive(smem_addr(full_b + u));
+      if (PAIR) {  // one arrival per warp, on the leader's barrier
+        __syncwarp();
+        if (lane == 0) {
+          if (q_rank == 0)
+            mbar_arrive(smem_addr(full_b + u));
+          else
+            mbar_arrive_remote(cluster_map(smem_addr(full_b + u), 0u));
+        }
+      } else {
+        mbar_arrive(smem_addr(full_b + u));
+      }
       return true;
     };
     static_assert(kStagesB == 3, "the dequantizing loop below is unrolled by three");
@@ -338,7 +460,10 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
   }
 
   // ---- accumulator ready?  (decided uniformly: tcgen05.ld is warp-collective)
-  const bool ready = warp < kDeqWarps ? mbar_wait_bounded(smem_addr(accum), 0) : true;
+  const bool ready =
+      warp < kDeqWarps
+          ? (PAIR ? mbar_wait_bounded(smem_addr(accum), 0) : mbar_wait_bounded(smem_addr(accum), 0))
+          : true;
   const int failed = __syncthreads_or(!ready || *abort_flag);
   tc_fence_after();
   if (failed && t == 0 && p.flag) *p.flag = AQNF4_ERR_TIMEOUT;
@@ -463,20 +588,31 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
       cluster_sync();
     }
   }
-  if (warp == kProducerWarp && lane == 0 && failed) {
+  if (warp == kProducerWarp && lane == 0 && failed && mma_cta) {
     // let every copy issued land before the shared memory goes away: tile s last received
-    // step s + kStagesA * ((issued - 1 - s) / kStagesA)
+    // step s + kStagesA * ((issued - 1 - s) / kStagesA).  (A pair's partner counts its copies
+    // on the leader's barriers, which it cannot wait on.  Its producer issues a copy only
+    // after the leader's MMAs released the tile, and the leader gives up only after a
+    // bounded wait of seconds on the missing copy, so nothing it issued is still in flight
+    // when the pair passes the barrier below.)
     for (int s = 0; s < kStagesA && s < issued; ++s)
       mbar_wait_bounded(smem_addr(full_a + s),
                         static_cast<uint32_t>((issued - 1 - s) / kStagesA) & 1);
   }
   tc_fence_before();
   __syncthreads();
+  // pair: neither CTA frees the TMEM or leaves while the other may still use its barriers
+  if (PAIR) cluster_sync();
   if (warp == kMmaWarp) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(kTmemCols)
-                 : "memory");
+    if (PAIR)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                   "r"(kTmemCols)
+                   : "memory");
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                   "r"(kTmemCols)
+                   : "memory");
   }
 }
 
@@ -512,26 +648,26 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// Whether a cluster of `splits` CTAs of this kernel can be resident at once (one CTA per SM:
-// it needs that many SMs of one GPC); asked once per device, kernel and size.
-bool cluster_fits(const void* kern, int splits) {
+// Whether a cluster of cx x cz CTAs of this kernel (cz = splits of K, or cx = 2 for a pair)
+// can be resident at once (one CTA per SM: it needs that many SMs of one GPC); asked once per
+// device, kernel and shape.
+bool cluster_fits(const void* kern, int which, int cx, int cz) {
   static std::mutex mu;
-  static int known[16][2][kMaxSplits + 1];  // 0 unknown, 1 fits, 2 does not
+  static int known[16][4][kMaxSplits + 1];  // 0 unknown, 1 fits, 2 does not
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return false;
-  const int which = kern == reinterpret_cast<const void*>(k_nf4_gemm<AQNF4_BF16>) ? 0 : 1;
   std::lock_guard<std::mutex> lock(mu);
-  int& k = known[dev][which][splits];
+  int& k = known[dev][which][cx * cz];
   if (k == 0) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(1, 1, static_cast<unsigned>(splits));
+    cfg.gridDim = dim3(static_cast<unsigned>(cx), 1, static_cast<unsigned>(cz));
     cfg.blockDim = dim3(kGThreads);
     cfg.dynamicSmemBytes = kGSmemBytes;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(cx);
     attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = static_cast<unsigned>(splits);
+    attr[0].val.clusterDim.z = static_cast<unsigned>(cz);
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int clusters = 0;
@@ -541,31 +677,53 @@ bool cluster_fits(const void* kern, int splits) {
   return k == 1;
 }
 
-template <int DT>
-cudaError_t launch_gemm(const CUtensorMap& map, const GParams& p, cudaStream_t stream) {
-  auto kern = k_nf4_gemm<DT>;
-  cudaError_t err =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmemBytes);
-  if (err != cudaSuccess) return err;
-  GParams q = p;
-  if (q.splits > 1 && !cluster_fits(reinterpret_cast<const void*>(kern), q.splits)) q.splits = 1;
-  const dim3 grid(static_cast<unsigned>((p.N + kBN - 1) / kBN),
-                  static_cast<unsigned>((p.M + kBM - 1) / kBM), static_cast<unsigned>(q.splits));
+template <int DT, bool PAIR>
+cudaError_t launch_cluster(const CUtensorMap& map, const GParams& q, unsigned row_tiles,
+                           cudaStream_t stream) {
+  auto kern = k_nf4_gemm<DT, PAIR>;
+  const unsigned col_tiles = static_cast<unsigned>((q.N + kBN - 1) / kBN);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
+  cfg.gridDim = PAIR ? dim3(row_tiles * col_tiles, 1, 1)  // row_tiles even
+                     : dim3(col_tiles, row_tiles, static_cast<unsigned>(q.splits));
   cfg.blockDim = dim3(kGThreads);
   cfg.dynamicSmemBytes = kGSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;  // the splits of a tile: one cluster
-  attr[0].val.clusterDim.x = 1;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = PAIR ? 2u : 1u;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = static_cast<unsigned>(q.splits);
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  err = cudaLaunchKernelEx(&cfg, kern, map, q);
+  const cudaError_t err = cudaLaunchKernelEx(&cfg, kern, map, q);
   count_launches(1);
   return err;
+}
+
+// Three launch forms: K split over a cluster of the tile's CTAs (few tiles); two row tiles
+// on a CTA pair with two-CTA MMAs (several row tiles, no split); or one CTA per tile.
+template <int DT>
+cudaError_t launch_gemm(const CUtensorMap& map, const GParams& p, cudaStream_t stream) {
+  auto single = k_nf4_gemm<DT, false>;
+  auto paired = k_nf4_gemm<DT, true>;
+  cudaError_t err =
+      cudaFuncSetAttribute(single, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmemBytes);
+  if (err == cudaSuccess)
+    err = cudaFuncSetAttribute(paired, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmemBytes);
+  if (err != cudaSuccess) return err;
+  const int wd = DT == AQNF4_BF16 ? 0 : 1;
+  GParams q = p;
+  const int64_t row_tiles = (p.M + kBM - 1) / kBM;
+  if (q.splits > 1 && !cluster_fits(reinterpret_cast<const void*>(single), wd, 1, q.splits))
+    q.splits = 1;
+  // a pair needs two row tiles (an odd count is rounded up: the last partner's rows are
+  // past M, its x copies read the fill value and its epilogue stores nothing)
+  const int64_t pair_ctas = (row_tiles + (row_tiles & 1)) * ((p.N + kBN - 1) / kBN);
+  if (q.splits == 1 && row_tiles >= 2 && pair_ctas <= INT32_MAX &&
+      cluster_fits(reinterpret_cast<const void*>(paired), 2 + wd, 2, 1))
+    return launch_cluster<DT, true>(map, q, static_cast<unsigned>(row_tiles + (row_tiles & 1)),
+                                    stream);
+  return launch_cluster<DT, false>(map, q, static_cast<unsigned>(row_tiles), stream);
 }
 
 }  // namespace
