@@ -62,6 +62,20 @@ constexpr uint32_t kTmemCols = 512;  // two f32 accumulators of 256 columns: all
 constexpr int kMaxSplits = 8;
 constexpr int kStageBytes = 128 * kBN * 4;
 static_assert(kStageBytes <= kBarBase, "the staged accumulator fits in the rings");
+
+// Ring geometry of each form.  A CTA pair's w_hat tile is half as large (128 rows), which
+// leaves room for a fourth x tile and a fourth w_hat tile in the same shared memory.
+template <bool PAIR>
+struct Ring {
+  static constexpr int SA = PAIR ? 4 : kStagesA;                     // x tiles
+  static constexpr int SB = PAIR ? 4 : kStagesB;                     // w_hat tiles
+  static constexpr int TB = (PAIR ? kBN / 2 : kBN) * kBK * 2;        // bytes of a w_hat tile
+  static constexpr int RingB = SA * kTileBytesA;                     // w_hat ring offset
+  static constexpr int BarBase = RingB + SB * TB;                    // barriers
+  static constexpr int FracOff = BarBase + 256;                      // fl(c / 255) table
+  static_assert(FracOff + 1024 + 1024 <= kGSmemBytes, "both forms fit the same allocation");
+  static_assert(2 * (SA + SB) * 8 + 8 + 16 <= 256, "the barriers fit their region");
+};
 static_assert(kDeqWarps * 16 == kBN, "two dequantizing threads per row of the w_hat tile");
 
 struct GParams {
@@ -221,6 +235,9 @@ template <int DT, bool PAIR>
 __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant__ CUtensorMap tmap_x,
                                                            const __grid_constant__ GParams p) {
   using F = Fmt<DT>;
+  using G = Ring<PAIR>;
+  constexpr int kStagesA = G::SA, kStagesB = G::SB, kTileBytesB = G::TB, kRingB = G::RingB,
+                kBarBase = G::BarBase, kFracOff = G::FracOff;
   extern __shared__ uint8_t smem_raw[];
   // the swizzled tiles need 1024-byte alignment
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -379,7 +396,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
     // w_hat tile (pair: CTA q holds rows n0 + 128 q + r, r < 128, at tile row r; threads
     // 4r .. 4r + 3 own its four quarters).  Step i's packed codes (16 or 8 bytes), 8-bit
     // constant and DQ scale are loaded from global memory while steps i - 3 .. i - 1 are
-    // worked on; the loop is unrolled by kStagesB (= 3), so step i + u always uses w_hat tile
+    // worked on; the loop is unrolled by kStagesB, so step i + u always uses w_hat tile
     // u and register set u.
     constexpr int kWords = PAIR ? 2 : 4;  // 32-bit words of packed codes per thread and step
     const float tab_level = p.level[lane & 15];  // lanes 16..31 mirror 0..15
@@ -442,20 +459,29 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
       }
       return true;
     };
-    static_assert(kStagesB == 3, "the dequantizing loop below is unrolled by three");
-    uint4 pk0 = make_uint4(0, 0, 0, 0), pk1 = pk0, pk2 = pk0;
-    uint32_t c0 = 0, c1 = 0, c2 = 0;
-    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f;
-    fetch(kt0, pk0, c0, s0);
-    fetch(kt0 + 1, pk1, c1, s1);
-    fetch(kt0 + 2, pk2, c2, s2);
-    for (int64_t i = 0; i < nk; i += 3) {
-      if (!dequant(i, 0, pk0, c0, s0)) break;
-      fetch(kt0 + i + 3, pk0, c0, s0);
-      if (i + 1 >= nk || !dequant(i + 1, 1, pk1, c1, s1)) break;
-      fetch(kt0 + i + 4, pk1, c1, s1);
-      if (i + 2 >= nk || !dequant(i + 2, 2, pk2, c2, s2)) break;
-      fetch(kt0 + i + 5, pk2, c2, s2);
+    // register set u (fully unrolled, so it stays in registers) holds step i + u's inputs
+    uint4 pkr[kStagesB];
+    uint32_t cr[kStagesB];
+    float sr[kStagesB];
+#pragma unroll
+    for (int u = 0; u < kStagesB; ++u) {
+      pkr[u] = make_uint4(0, 0, 0, 0);
+      cr[u] = 0;
+      sr[u] = 0.0f;
+      fetch(kt0 + u, pkr[u], cr[u], sr[u]);
+    }
+    bool going = true;
+    for (int64_t i = 0; i < nk && going; i += kStagesB) {
+#pragma unroll
+      for (int u = 0; u < kStagesB; ++u) {
+        if (going) {
+          if (i + u >= nk || !dequant(i + u, u, pkr[u], cr[u], sr[u])) {
+            going = false;
+          } else {
+            fetch(kt0 + i + u + kStagesB, pkr[u], cr[u], sr[u]);
+          }
+        }
+      }
     }
   }
 
