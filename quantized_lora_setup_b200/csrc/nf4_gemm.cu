@@ -280,8 +280,9 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
       mbar_init(smem_addr(empty_a + s), 1);
     }
     for (int s = 0; s < kStagesB; ++s) {
-      // pair: one arrival per dequantizing warp of either CTA, on the leader's barrier
-      mbar_init(smem_addr(full_b + s), PAIR ? 2 * kDeqWarps : 32 * kDeqWarps);
+      // pair: one arrival per dequantizing warp of the tile's group in either CTA, on the
+      // leader's barrier
+      mbar_init(smem_addr(full_b + s), PAIR ? kDeqWarps : 32 * kDeqWarps);
       mbar_init(smem_addr(empty_b + s), 1);
     }
     mbar_init(smem_addr(accum), 1);
@@ -393,27 +394,26 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
     }
   } else {
     // ---- dequantizing warps: threads 2r and 2r + 1 own the two halves of row n0 + r of the
-    // w_hat tile (pair: CTA q holds rows n0 + 128 q + r, r < 128, at tile row r; threads
-    // 4r .. 4r + 3 own its four quarters).  Step i's packed codes (16 or 8 bytes), 8-bit
-    // constant and DQ scale are loaded from global memory while steps i - 3 .. i - 1 are
-    // worked on; the loop is unrolled by kStagesB, so step i + u always uses w_hat tile
-    // u and register set u.
-    constexpr int kWords = PAIR ? 2 : 4;  // 32-bit words of packed codes per thread and step
+    // w_hat tile.  A pair's CTA q holds rows n0 + 128 q + r (r < 128) at tile row r, and its
+    // dequantizing warps form two groups of eight that take alternate steps (group g: steps
+    // i = g mod 2), so each thread still rebuilds 32 elements per step it takes.  Step i's
+    // 16 bytes of packed codes, 8-bit constant and DQ scale are loaded from global memory
+    // kStagesB steps ahead; the loop is unrolled over the group's register sets, one per
+    // w_hat tile the group uses.
+    constexpr int kGroups = PAIR ? 2 : 1;
+    constexpr int kSets = kStagesB / kGroups;
+    static_assert(kSets * kGroups == kStagesB, "each group owns whole w_hat tiles");
+    const int grp = PAIR ? warp >> 3 : 0;
+    const int tg = t - grp * (32 * kDeqWarps / kGroups);  // thread within its group
     const float tab_level = p.level[lane & 15];  // lanes 16..31 mirror 0..15
-    const int r = PAIR ? t >> 2 : t >> 1;
-    const int part = PAIR ? (t & 3) : (t & 1);
+    const int r = tg >> 1, hf = tg & 1;
     const int64_t n = n0 + 128 * static_cast<int64_t>(q_rank) + r;
     const bool row_ok = n < p.N;
-    const uint8_t* prow = p.packed + n * (p.K / 2) + part * (4 * kWords);
+    const uint8_t* prow = p.packed + n * (p.K / 2) + hf * 16;
     auto fetch = [&](int64_t kt, uint4& pk, uint32_t& c, float& s8) {
       if (row_ok && kt < kt1) {
         const int64_t b = n * kb + kt;
-        if (PAIR) {
-          const uint2 v = __ldg(reinterpret_cast<const uint2*>(prow + kt * (kBK / 2)));
-          pk = make_uint4(v.x, v.y, 0u, 0u);
-        } else {
-          pk = __ldg(reinterpret_cast<const uint4*>(prow + kt * (kBK / 2)));
-        }
+        pk = __ldg(reinterpret_cast<const uint4*>(prow + kt * (kBK / 2)));
         c = __ldg(p.codes8 + b);
         s8 = __ldg(p.scales + (b >> 8));
       }
@@ -421,8 +421,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
     // one step into w_hat tile u; false when the pipeline has been aborted
     auto dequant = [&](int64_t i, int u, const uint4& pk, uint32_t c8, float sc) -> bool {
       const uint32_t par = static_cast<uint32_t>(i / kStagesB - 1) & 1;
-      bool ok = i < kStagesB || (PAIR ? mbar_wait_bounded(smem_addr(empty_b + u), par)
-                                      : mbar_wait_bounded(smem_addr(empty_b + u), par));
+      bool ok = i < kStagesB || mbar_wait_bounded(smem_addr(empty_b + u), par);
       if (!ok) *abort_flag = 1;
       if (__any_sync(kFull, *abort_flag != 0)) return false;  // warp-uniform (shuffles below)
       // a zero constant (also for rows past N) gives 0
@@ -431,7 +430,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
       const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
       uint8_t* rowb = smem + kRingB + u * kTileBytesB + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-      for (int jj = 0; jj < kWords; ++jj) {
+      for (int jj = 0; jj < 4; ++jj) {
         const uint32_t w = words[jj];
         uint32_t o[4];
 #pragma unroll
@@ -442,7 +441,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
           const f32x2 v = pmul_rn(pair(q0, q1), a2);
           o[h] = F::pack_rn(pair_lo(v), pair_hi(v));
         }
-        const int j = kWords * part + jj;  // 16-byte chunk of the 128-byte row
+        const int j = 4 * hf + jj;  // 16-byte chunk of the 128-byte row
         *reinterpret_cast<uint4*>(rowb + ((j ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
       }
       fence_proxy_async_smem();  // the tensor cores read this tile through the async proxy
@@ -459,26 +458,29 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
       }
       return true;
     };
-    // register set u (fully unrolled, so it stays in registers) holds step i + u's inputs
-    uint4 pkr[kStagesB];
-    uint32_t cr[kStagesB];
-    float sr[kStagesB];
+    // register set v (fully unrolled, so it stays in registers) holds the inputs of the
+    // group's step that uses w_hat tile u = v kGroups + grp
+    uint4 pkr[kSets];
+    uint32_t cr[kSets];
+    float sr[kSets];
 #pragma unroll
-    for (int u = 0; u < kStagesB; ++u) {
-      pkr[u] = make_uint4(0, 0, 0, 0);
-      cr[u] = 0;
-      sr[u] = 0.0f;
-      fetch(kt0 + u, pkr[u], cr[u], sr[u]);
+    for (int v = 0; v < kSets; ++v) {
+      pkr[v] = make_uint4(0, 0, 0, 0);
+      cr[v] = 0;
+      sr[v] = 0.0f;
+      fetch(kt0 + v * kGroups + grp, pkr[v], cr[v], sr[v]);
     }
     bool going = true;
-    for (int64_t i = 0; i < nk && going; i += kStagesB) {
+    for (int64_t i0 = 0; i0 < nk && going; i0 += kStagesB) {
 #pragma unroll
-      for (int u = 0; u < kStagesB; ++u) {
+      for (int v = 0; v < kSets; ++v) {
+        const int u = v * kGroups + grp;
+        const int64_t i = i0 + u;
         if (going) {
-          if (i + u >= nk || !dequant(i + u, u, pkr[u], cr[u], sr[u])) {
+          if (i >= nk || !dequant(i, u, pkr[v], cr[v], sr[v])) {
             going = false;
           } else {
-            fetch(kt0 + i + u + kStagesB, pkr[u], cr[u], sr[u]);
+            fetch(kt0 + i + kStagesB, pkr[v], cr[v], sr[v]);
           }
         }
       }
