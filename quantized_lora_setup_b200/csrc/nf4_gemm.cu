@@ -49,6 +49,10 @@ constexpr int kBM = 256, kBN = 256, kBK = 64;  // two 128-row accumulators
 // on-chip memory to the L1 that serves the dequantizing warps' global loads.
 constexpr int kStagesA = 3, kStagesB = 3;
 constexpr int kDeqWarps = 16, kProducerWarp = 16, kMmaWarp = 17;
+// A CTA pair's dequantizing warps take the steps in four groups of four warps, in turn: a
+// thread rebuilds a whole 64-element row of its half of the w_hat tile every fourth step,
+// so the per-step costs (waits, loads, the arrival) are paid once per 64 elements.
+constexpr int kPairGroups = 4;
 constexpr int kGThreads = 32 * (kDeqWarps + 2);            // 576
 constexpr int kTileBytesA = kBM * kBK * 2;                  // 32 KB of x
 constexpr int kTileBytesB = kBN * kBK * 2;                  // 32 KB of w_hat
@@ -282,7 +286,7 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
     for (int s = 0; s < kStagesB; ++s) {
       // pair: one arrival per dequantizing warp of the tile's group in either CTA, on the
       // leader's barrier
-      mbar_init(smem_addr(full_b + s), PAIR ? kDeqWarps : 32 * kDeqWarps);
+      mbar_init(smem_addr(full_b + s), PAIR ? 2 * kDeqWarps / kPairGroups : 32 * kDeqWarps);
       mbar_init(smem_addr(empty_b + s), 1);
     }
     mbar_init(smem_addr(accum), 1);
@@ -395,31 +399,37 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
   } else {
     // ---- dequantizing warps: threads 2r and 2r + 1 own the two halves of row n0 + r of the
     // w_hat tile.  A pair's CTA q holds rows n0 + 128 q + r (r < 128) at tile row r, and its
-    // dequantizing warps form two groups of eight that take alternate steps (group g: steps
-    // i = g mod 2), so each thread still rebuilds 32 elements per step it takes.  Step i's
-    // 16 bytes of packed codes, 8-bit constant and DQ scale are loaded from global memory
-    // kStagesB steps ahead; the loop is unrolled over the group's register sets, one per
-    // w_hat tile the group uses.
-    constexpr int kGroups = PAIR ? 2 : 1;
+    // dequantizing warps form kPairGroups groups that take the steps in turn (group g: steps
+    // i = g mod kPairGroups); thread r of a group rebuilds all of row r.  Step i's packed
+    // codes, 8-bit constant and DQ scale are loaded from global memory kStagesB steps ahead;
+    // the loop is unrolled over the group's register sets, one per w_hat tile it uses.
+    constexpr int kGroups = PAIR ? kPairGroups : 1;
     constexpr int kSets = kStagesB / kGroups;
     static_assert(kSets * kGroups == kStagesB, "each group owns whole w_hat tiles");
-    const int grp = PAIR ? warp >> 3 : 0;
+    constexpr int kTpr = PAIR && kGroups == 4 ? 1 : 2;  // threads per w_hat row
+    constexpr int kVec = 2 / kTpr;                      // 16-byte code loads per thread and step
+    const int grp = warp / (kDeqWarps / kGroups);
     const int tg = t - grp * (32 * kDeqWarps / kGroups);  // thread within its group
     const float tab_level = p.level[lane & 15];  // lanes 16..31 mirror 0..15
-    const int r = tg >> 1, hf = tg & 1;
+    const int r = tg / kTpr, hf = tg % kTpr;
     const int64_t n = n0 + 128 * static_cast<int64_t>(q_rank) + r;
     const bool row_ok = n < p.N;
     const uint8_t* prow = p.packed + n * (p.K / 2) + hf * 16;
-    auto fetch = [&](int64_t kt, uint4& pk, uint32_t& c, float& s8) {
+    struct Codes {
+      uint4 v[kVec];
+    };
+    auto fetch = [&](int64_t kt, Codes& pk, uint32_t& c, float& s8) {
       if (row_ok && kt < kt1) {
         const int64_t b = n * kb + kt;
-        pk = __ldg(reinterpret_cast<const uint4*>(prow + kt * (kBK / 2)));
+#pragma unroll
+        for (int k = 0; k < kVec; ++k)
+          pk.v[k] = __ldg(reinterpret_cast<const uint4*>(prow + kt * (kBK / 2) + 16 * k));
         c = __ldg(p.codes8 + b);
         s8 = __ldg(p.scales + (b >> 8));
       }
     };
     // one step into w_hat tile u; false when the pipeline has been aborted
-    auto dequant = [&](int64_t i, int u, const uint4& pk, uint32_t c8, float sc) -> bool {
+    auto dequant = [&](int64_t i, int u, const Codes& pk, uint32_t c8, float sc) -> bool {
       const uint32_t par = static_cast<uint32_t>(i / kStagesB - 1) & 1;
       bool ok = i < kStagesB || mbar_wait_bounded(smem_addr(empty_b + u), par);
       if (!ok) *abort_flag = 1;
@@ -427,10 +437,17 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
       // a zero constant (also for rows past N) gives 0
       const float ap = row_ok ? __fmul_rn(frac[c8], sc) : 0.0f;
       const f32x2 a2 = pair(ap, ap);
-      const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
+      uint32_t words[4 * kVec];
+#pragma unroll
+      for (int k = 0; k < kVec; ++k) {
+        words[4 * k] = pk.v[k].x;
+        words[4 * k + 1] = pk.v[k].y;
+        words[4 * k + 2] = pk.v[k].z;
+        words[4 * k + 3] = pk.v[k].w;
+      }
       uint8_t* rowb = smem + kRingB + u * kTileBytesB + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
+      for (int jj = 0; jj < 4 * kVec; ++jj) {
         const uint32_t w = words[jj];
         uint32_t o[4];
 #pragma unroll
@@ -460,12 +477,13 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
     };
     // register set v (fully unrolled, so it stays in registers) holds the inputs of the
     // group's step that uses w_hat tile u = v kGroups + grp
-    uint4 pkr[kSets];
+    Codes pkr[kSets];
     uint32_t cr[kSets];
     float sr[kSets];
 #pragma unroll
     for (int v = 0; v < kSets; ++v) {
-      pkr[v] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int k = 0; k < kVec; ++k) pkr[v].v[k] = make_uint4(0, 0, 0, 0);
       cr[v] = 0;
       sr[v] = 0.0f;
       fetch(kt0 + v * kGroups + grp, pkr[v], cr[v], sr[v]);
