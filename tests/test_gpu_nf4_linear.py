@@ -44,8 +44,9 @@ def _run(cuda, x, packed, codes8, scales, N, out_dtype):
                                    (70, 260, 320), (600, 300, 256), (520, 1000, 512),
                                    (1024, 512, 960)])
 def test_nf4_linear_matches_oracle(cuda, dt, M, N, K):
-    """Shapes with one CTA per tile (several row tiles, an odd count: 600 and 520 rows) and
-    with split K."""
+    """Shapes with one CTA per tile, with split K, and with two row tiles per CTA pair
+    (several row tiles and no split: 600, 520 and 1024 rows; an odd count of row tiles
+    leaves the last pair's second CTA without rows)."""
     x, packed, codes8, scales = _case(M, N, K, dt, seed=M + N + K)
     ref, rabs = oracle.nf4_linear(synth.bits_u16(x).reshape(M, K), DT[dt], packed, codes8,
                                   scales, N, DT[dt])
@@ -86,9 +87,9 @@ def test_nf4_linear_split_k_matches_oracle(cuda, dt, M, N, K, S):
 
 @pytest.mark.gpu
 def test_nf4_linear_full_mlp_shape_sampled_rows(cuda):
-    """The 7B MLP up-projection at 4096 tokens (11008 x 4096, bf16), as the bench times it:
-    rows of y from several row tiles and both 128-row halves of a tile, against the
-    oracle's product of those rows of x."""
+    """The 7B MLP up-projection at 4096 tokens (11008 x 4096, bf16; CTA pairs with two-CTA
+    MMAs), as the bench times it: rows of y from several row tiles, from both CTAs of a pair
+    and from both 128-row halves of a tile, against the oracle's product of those rows."""
     M, N, K = 4096, 11008, 4096
     x, packed, codes8, scales = _case(M, N, K, torch.bfloat16, seed=11)
     y = torch.full((M, N), float("nan"), dtype=torch.float32, device=cuda)
