@@ -311,6 +311,29 @@ def test_dequantize_matches_oracle(cuda, out_dt, n):
     assert np.array_equal(bits(got2.cpu()), ref2)
 
 
+@pytest.mark.parametrize("out_dt", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("n", [9, 65, 1023, 16384 + 3, 200001])
+def test_dequantize_16_byte_aligned_output(cuda, out_dt, n):
+    """An output that is 16- but not 32-byte aligned takes the 16-byte-store path (an
+    aligned one the 32-byte-store path, above); both, plain and mean-centred, equal the
+    oracle bit for bit, and the 16 bytes in front of the output stay untouched."""
+    w = synth.random_bits_host(n, seed=n + 23, dtype=torch.bfloat16)
+    op, oa, _ = oracle.quantize(bits(w), oracle.BF16)
+    oc, osc, _ = oracle.double_quant(oa)
+    cc, csc, cmu, _ = oracle.double_quant_centered(oa)
+    dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).to(cuda)
+    buf = torch.full((n + 8,), 7, dtype=out_dt, device=cuda)  # 256-byte aligned allocation
+    out = buf[8:]  # 16 bytes in: aligned to 16 bytes, not to 32
+    assert out.data_ptr() % 32 == 16
+    aqnf4.aqnf4_dequantize(dev(op), dev(oc), dev(osc), None, n, out)
+    assert np.array_equal(bits(out.cpu()), oracle.dequantize(op, n, DT[out_dt], codes8=oc,
+                                                            scales=osc))
+    aqnf4.aqnf4_dequantize_centered(dev(op), dev(cc), dev(csc), dev(cmu), n, out)
+    assert np.array_equal(bits(out.cpu()), oracle.dequantize_centered(op, n, DT[out_dt], cc,
+                                                                     csc, cmu))
+    assert torch.equal(buf[:8].cpu(), torch.full((8,), 7, dtype=out_dt))
+
+
 @pytest.mark.parametrize("seed", range(8))
 def test_select_topk_matches_oracle(cuda, seed):
     rng = np.random.default_rng(seed)
