@@ -230,7 +230,8 @@ AQNF4_API aqnf4_status aqnf4_layer_error_noalloc(const aqnf4_layer* layers, int3
    the layer is whole NF4 blocks.  When the output has too few 256 x 256 tiles to fill the
    GPU, K is split over aqnf4_nf4_linear_splits(M, N, K) thread blocks that form one cluster
    per tile and add their binary32 partial sums on chip, in split order (the result does not
-   depend on scheduling, and no workspace is needed).  dev_flag (optional, device int32)
+   depend on scheduling, and no workspace is needed).  Otherwise, with more than 256 rows,
+   two row tiles share each dequantized weight tile on a pair of thread blocks.  dev_flag (optional, device int32)
    receives AQNF4_ERR_TIMEOUT if a bounded wait inside the kernel gave up; the tiles that
    wait belonged to are then not written (without a dev_flag a timeout goes unreported and y
    is undefined).
