@@ -230,6 +230,11 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
       : "memory");
 }
 
+// barrier over the dequantizing warps alone (named barrier 1)
+__device__ __forceinline__ void deq_bar_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * kDeqWarps) : "memory");
+}
+
 // arrival on a barrier of another CTA of the cluster
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
@@ -514,39 +519,68 @@ __global__ void __launch_bounds__(kGThreads, 1) k_nf4_gemm(const __grid_constant
   tc_fence_after();
   if (failed && t == 0 && p.flag) *p.flag = AQNF4_ERR_TIMEOUT;
   if (p.splits == 1 && !failed && warp < kDeqWarps) {
-    // warp w: TMEM lanes 32 (w mod 4).. ; accumulator (w / 8) holds rows 128 (w / 8).. of the
-    // tile; columns 128 ((w / 4) mod 2)..
-    const int q = warp & 3, acc = warp >> 3, chalf = (warp >> 2) & 1;
-    const int64_t m = m0 + 128 * acc + 32 * q + lane;
+    // y, one 128-row accumulator at a time, through the (now idle) rings: warp w reads TMEM
+    // lanes 32 (w mod 4).. (rows) and columns 64 (w / 4).., converts to y's format and stages
+    // the rows in shared memory (16-byte chunk j of row r at j ^ (r mod 8): neither these
+    // stores nor the reads below conflict on banks); then each warp writes whole rows of the
+    // tile, 512 or 1024 contiguous bytes per row, rows w, w + 16, ..  The dequantizing warps
+    // alone take part (named barrier 1); the staging needs 128 x 256 x 4 bytes at most.
+    static_assert(128 * kBN * 4 <= Ring<PAIR>::BarBase, "a staged accumulator fits in the rings");
+    const bool f32o = p.out_f32 != 0;
+    const int esz = f32o ? 4 : 2;
+    const int row_bytes = kBN * esz;    // 1024 or 512
+    const int per = 16 / esz;           // elements per 16-byte chunk
+    const int chunks = row_bytes / 16;  // 64 or 32 per row
+    const bool vec = f32o ? (p.N & 3) == 0 : (p.N & 7) == 0;  // 16-byte aligned rows of y
+    const int q = warp & 3, cq = warp >> 2;
+    const int rr = 32 * q + lane;
+    for (int hh = 0; hh < (lower_half ? 2 : 1); ++hh) {
+      if (hh > 0) deq_bar_sync();  // the first half's rows have been read out
+      uint8_t* srow = smem + rr * row_bytes;
 #pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      float v[32];
-      const int cbase = 128 * chalf + 32 * c;
-      tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + kBN * acc + cbase, v);
-      const int64_t col = n0 + cbase;
-      if (m < p.M && col < p.N) {
-        const bool whole = col + 32 <= p.N;
-        if (p.out_f32) {
-          float* dst = static_cast<float*>(p.y) + m * p.N + col;
-          if (whole && (p.N & 3) == 0) {
+      for (int c = 0; c < 2; ++c) {
+        float v[32];
+        const int cbase = 64 * cq + 32 * c;
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q) << 16) + kBN * hh + cbase, v);
+        if (f32o) {
 #pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              *reinterpret_cast<float4*>(dst + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-          } else {
-            for (int i = 0; i < 32 && col + i < p.N; ++i) dst[i] = v[i];
+          for (int i = 0; i < 8; ++i) {
+            const int j = cbase / 4 + i;
+            *reinterpret_cast<float4*>(srow + ((j ^ (rr & 7)) << 4)) =
+                make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
           }
         } else {
-          uint16_t* dst = static_cast<uint16_t*>(p.y) + m * p.N + col;
-          uint32_t h[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) h[i] = F::pack_rn(v[2 * i], v[2 * i + 1]);
-          if (whole && (p.N & 7) == 0) {
-#pragma unroll
-            for (int i = 0; i < 16; i += 4)
-              *reinterpret_cast<uint4*>(dst + 2 * i) = make_uint4(h[i], h[i + 1], h[i + 2], h[i + 3]);
+          for (int i = 0; i < 4; ++i) {
+            const int j = cbase / 8 + i;
+            *reinterpret_cast<uint4*>(srow + ((j ^ (rr & 7)) << 4)) = make_uint4(
+                F::pack_rn(v[8 * i], v[8 * i + 1]), F::pack_rn(v[8 * i + 2], v[8 * i + 3]),
+                F::pack_rn(v[8 * i + 4], v[8 * i + 5]), F::pack_rn(v[8 * i + 6], v[8 * i + 7]));
+          }
+        }
+      }
+      deq_bar_sync();  // the half is staged
+#pragma unroll 1
+      for (int k = 0; k < 128 / kDeqWarps; ++k) {
+        const int r2 = warp + kDeqWarps * k;
+        const int64_t m = m0 + 128 * hh + r2;
+        if (m >= p.M) break;  // warp-uniform; later rows lie further down
+        for (int j = lane; j < chunks; j += 32) {
+          const uint4 val = lds128(smem + r2 * row_bytes + ((j ^ (r2 & 7)) << 4));
+          const int64_t col = n0 + static_cast<int64_t>(j) * per;
+          if (col >= p.N) continue;
+          uint8_t* dst = static_cast<uint8_t*>(p.y) + (m * p.N + col) * esz;
+          if (vec && col + per <= p.N) {
+            *reinterpret_cast<uint4*>(dst) = val;
           } else {
-            for (int i = 0; i < 32 && col + i < p.N; ++i)
-              dst[i] = static_cast<uint16_t>(h[i >> 1] >> (16 * (i & 1)));
+            for (int e = 0; e < per && col + e < p.N; ++e) {
+              const int k = f32o ? e : e >> 1;  // the 32-bit word holding element e
+              const uint32_t w = k == 0 ? val.x : k == 1 ? val.y : k == 2 ? val.z : val.w;
+              if (f32o)
+                reinterpret_cast<uint32_t*>(dst)[e] = w;
+              else
+                reinterpret_cast<uint16_t*>(dst)[e] = static_cast<uint16_t>(w >> (16 * (e & 1)));
+            }
           }
         }
       }
