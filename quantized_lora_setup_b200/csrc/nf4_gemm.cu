@@ -14,23 +14,24 @@
 //   - warps 0-15 dequantize the step's 256-row slice of the layer into a 256 x 64 w_hat tile
 //     (one of kStagesB) -- threads 2r and 2r + 1 take the two halves of row n0 + r, one NF4
 //     block per row and step (K is a multiple of 64) -- in the same swizzled K-major layout,
-//     16 bytes at a time, and arrive on the tile's barrier.  Each thread loads its 16 bytes of
-//     packed codes, the block's 8-bit constant and its DQ scale from global memory three
-//     steps ahead into registers, so a w_hat tile can be rebuilt as soon as the tensor cores
+//     16 bytes at a time, and arrive on the tile's barrier.  Each thread loads its packed
+//     codes, the block's 8-bit constant and its DQ scale from global memory kStagesB steps
+//     ahead into registers, so a w_hat tile can be rebuilt as soon as the tensor cores
 //     release it, without waiting for a copy;
 //   - warp 17 issues eight tcgen05.mma per step (M 128, N 256, K 16, bf16/f16 in, f32 out):
 //     each x row half against the same w_hat tile, into two TMEM accumulators that fill all
 //     512 columns, so every dequantized element feeds 256 rows of x; tcgen05.commit frees
 //     the stage when they finish;
-//   - warps 0-15 then read the accumulators with tcgen05.ld (warp w: TMEM lanes 32(w mod 4)..,
-//     accumulator w / 8, columns 128 ((w / 4) mod 2)..) and store y.
+//   - warps 0-15 then read the accumulators with tcgen05.ld, stage each 128-row accumulator
+//     in the idle rings and write y in whole rows.
 // When the output has too few tiles to fill the GPU, K is split over up to 8 CTAs that form
 // one thread-block cluster per tile; they add their partial sums through distributed shared
 // memory instead of a trip through HBM and a second kernel.  With two or more row tiles and
 // no split, two row tiles run on a CTA pair with two-CTA MMAs (tcgen05.mma.cta_group::2,
 // M = 256 of which 128 rows from each CTA, N = 256 of which each CTA holds and dequantizes
 // 128 w_hat rows): each CTA rebuilds half the w_hat tile, and the tensor cores read a
-// w_hat row from shared memory once per 512 rows of x instead of once per 128.
+// w_hat row from shared memory once per 512 rows of x instead of once per 128.  A pair's
+// dequantizing warps work in four groups that take the steps in turn, one thread per row.
 // Every wait is bounded: a wait that gives up records AQNF4_ERR_TIMEOUT and makes every role
 // stop; copies in flight are allowed to land and the TMEM is always freed before exit.
 #include <cuda.h>
