@@ -506,11 +506,12 @@ def run_only_nf4_linear(args):
     return 0
 
 
-def bench_nf4_linear(dev, stream, reps=20, shapes=((4096, 11008, 4096), (128, 11008, 4096)),
+def bench_nf4_linear(dev, stream, reps=20,
+                     shapes=((4096, 11008, 4096), (512, 11008, 4096), (128, 11008, 4096)),
                      baseline=True):
     """The forward product of an NF4 + DQ layer, y = x w_hat^T, with the dequantization fused
     into the tcgen05 GEMM (aqnf4_nf4_linear): the 7B-shaped MLP up-projection (11008 x 4096)
-    at 4096 and 128 tokens, bf16.  TFLOP/s against the measured bf16 peak, beside the unfused
+    at 4096, 512 and 128 tokens, bf16.  TFLOP/s against the measured bf16 peak, beside the unfused
     path (aqnf4_dequantize, then cuBLAS on the bf16 weights) for context."""
     import torch
 

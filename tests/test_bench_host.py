@@ -70,6 +70,7 @@ def test_compact_summary_fits_the_line_tail(bench):
                                                 "packed_1024MB")]},
          "nf4_linear": {"unit": "TFLOP/s", "tokens_4096": {"value": 1000.0,
                                                             "dequant_then_cublas": 1400.0},
+                        "tokens_512": {"value": 800.0, "dequant_then_cublas": 700.0},
                         "tokens_128": {"value": 260.0, "dequant_then_cublas": 280.0}},
          "dq_score": {"roofline": rf}}
     s = bench.compact_summary(r)
@@ -78,6 +79,6 @@ def test_compact_summary_fits_the_line_tail(bench):
     assert line.endswith(json.dumps(s) + "}")
     assert len(json.dumps(s)) < 1000
     for key in ("frac", "layers_per_s", "14b", "1.4b", "dequant", "gemm_tokens_4096",
-                "gemm_tokens_128", "dq_score_frac"):
+                "gemm_tokens_512", "gemm_tokens_128", "dq_score_frac"):
         assert key in s
     assert s["dequant"]["packed_8MB"] == [0.5, 0.6]
