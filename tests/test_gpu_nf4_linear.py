@@ -42,11 +42,13 @@ def _run(cuda, x, packed, codes8, scales, N, out_dtype):
 @pytest.mark.parametrize("M,N,K", [(128, 128, 64), (1, 1, 64), (200, 300, 256),
                                    (256, 384, 4096), (130, 129, 192), (64, 100, 128),
                                    (70, 260, 320), (600, 300, 256), (520, 1000, 512),
-                                   (1024, 512, 960), (300, 1001, 448)])
+                                   (1024, 512, 960), (300, 1001, 448), (257, 256, 64),
+                                   (300, 512, 192), (513, 384, 320)])
 def test_nf4_linear_matches_oracle(cuda, dt, M, N, K):
     """Shapes with one CTA per tile, with split K, and with two row tiles per CTA pair
     (several row tiles and no split: 600, 520 and 1024 rows; an odd count of row tiles
-    leaves the last pair's second CTA without rows)."""
+    leaves the last pair's second CTA without rows; 1, 3 or 5 steps of K leave some of
+    the pair's four dequantizing groups without a step)."""
     x, packed, codes8, scales = _case(M, N, K, dt, seed=M + N + K)
     ref, rabs = oracle.nf4_linear(synth.bits_u16(x).reshape(M, K), DT[dt], packed, codes8,
                                   scales, N, DT[dt])
