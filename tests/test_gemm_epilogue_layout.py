@@ -70,3 +70,37 @@ def replay(M, N, m0, n0, f32_out):
                                        (256, 256, 0, 0), (130, 129, 0, 0)])
 def test_staged_epilogue_writes_each_element_once(M, N, m0, n0, f32_out):
     replay(M, N, m0, n0, f32_out)
+
+
+def replay_split(M, N, m0, n0, S):
+    """Split K: after the first cluster barrier, CTA z of the S CTAs of a tile adds rows
+    [rows z / S, rows (z + 1) / S) of each staged 128-row accumulator (binary32, 1024-byte
+    rows, chunk j of row r at 16 (j ^ (r mod 8))); thread e of 576 takes (row lo + e / nch,
+    chunk e mod nch), 4 columns a chunk."""
+    threads = 576
+    cols = min(BN, N - n0)
+    nch = (cols + 3) // 4
+    written = {}
+    for hh in range(2 if m0 + 128 < M else 1):
+        rows = min(128, M - (m0 + 128 * hh))
+        for z in range(S):
+            lo, hi = rows * z // S, rows * (z + 1) // S
+            for t in range(threads):
+                for e in range(t, (hi - lo) * nch, threads):
+                    r, j = lo + e // nch, e % nch
+                    off = r * BN * 4 + ((j ^ (r & 7)) << 4)
+                    assert off + 16 <= 128 * 1024
+                    for k in range(4):
+                        if 4 * j + k < cols:
+                            key = (m0 + 128 * hh + r, n0 + 4 * j + k)
+                            assert key not in written
+                            written[key] = z
+    want = {(m, c) for m in range(m0, min(M, m0 + 256)) for c in range(n0, min(N, n0 + 256))}
+    assert set(written) == want
+
+
+@pytest.mark.parametrize("S", [2, 3, 4, 7, 8])
+@pytest.mark.parametrize("M,N,m0,n0", [(128, 11008, 0, 10752), (7, 1023, 0, 768),
+                                       (300, 512, 256, 256), (200, 10240, 0, 0)])
+def test_split_k_sum_covers_each_output_once(M, N, m0, n0, S):
+    replay_split(M, N, m0, n0, S)
