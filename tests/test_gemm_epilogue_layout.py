@@ -7,7 +7,7 @@ chunks l, l + 32, ..  This replays that index arithmetic on the CPU and checks t
 element of a tile inside M x N is written exactly once, from its own accumulator entry, for
 f32 and 16-bit outputs and ragged edges; that staging stays inside the 128 KB it may use; and
 that the eight lanes of each 16-byte shared-memory access phase hit eight different bank
-groups on both sides.
+groups on both sides.  The split-K sum's row slices and chunks are replayed the same way.
 """
 import pytest
 
